@@ -1,0 +1,133 @@
+"""Seeded synthetic inputs for the NVFP4 linear layer.
+
+This module holds no quantization arithmetic: it only draws bf16 tensors with the shapes and
+value distributions of the pretraining workloads the Quartet II pages describe (LLM linear
+layers: activations X [M,K], weights W [N,K] in PyTorch ``Linear`` layout, output gradients
+dY [M,N]).  Both the CUDA path's tests and the oracle's tests draw their inputs here, so the
+two sides see the same bytes.
+
+Recipes (seed s; X, W and dY use sub-seeds s, s+1, s+2):
+  tiny       X, W, dY 256x256, N(0,1); W scaled by 0.02.
+  llm1p9b    M=16384, K=2048, N=8192.  X = t_3/sqrt(3) with a seeded 4 of every 1024
+             channels (columns) scaled by 20; W ~ N(0, 0.02^2); dY ~ N(0, (1e-4)^2).
+  mlp8b_up   M=16384, K=4096, N=14336 (gate/up): X ~ N(0,1); W ~ N(0, 0.02^2);
+             dY = N(0, (1e-4)^2) * exp(z_m) with z_m ~ N(0,1) per row.
+  mlp8b_down M=16384, K=14336, N=4096: X = SiLU(a) * b with a, b ~ N(0,1); W, dY as above.
+  sweep      a bf16 [rows, L] tensor ~ N(0,1), each element independently x50 with p=0.001.
+"""
+from __future__ import annotations
+
+import torch
+
+SHAPES = {
+    "tiny": (256, 256, 256),
+    "llm1p9b": (16384, 2048, 8192),
+    "mlp8b_up": (16384, 4096, 14336),
+    "mlp8b_down": (16384, 14336, 4096),
+}
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, device) -> torch.Tensor:
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+
+def student_t3_unit(shape, g, device) -> torch.Tensor:
+    """Student-t with 3 degrees of freedom divided by sqrt(3) (unit variance):
+    Z / sqrt(chi2_3 / 3) / sqrt(3) = Z / sqrt(chi2_3)."""
+    z = _randn(shape, g, device)
+    chi2 = torch.zeros(shape, device=device, dtype=torch.float32)
+    for _ in range(3):
+        chi2 += _randn(shape, g, device) ** 2
+    return z / torch.sqrt(chi2)
+
+
+def make_x(M: int, K: int, kind: str, seed: int, device="cpu") -> torch.Tensor:
+    g = _gen(device, seed)
+    if kind == "gauss":
+        x = _randn((M, K), g, device)
+    elif kind == "t3_outlier_channels":
+        x = student_t3_unit((M, K), g, device)
+        n_out = max(1, (4 * K) // 1024)
+        perm = torch.randperm(K, generator=g, device=device)[:n_out]
+        x[:, perm] *= 20.0
+    elif kind == "silu_gated":
+        a = _randn((M, K), g, device)
+        b = _randn((M, K), g, device)
+        x = torch.nn.functional.silu(a) * b
+    else:
+        raise ValueError(kind)
+    return x.to(torch.bfloat16)
+
+
+def make_w(N: int, K: int, seed: int, std: float = 0.02, device="cpu") -> torch.Tensor:
+    g = _gen(device, seed)
+    return (_randn((N, K), g, device) * std).to(torch.bfloat16)
+
+
+def make_dy(M: int, N: int, kind: str, seed: int, device="cpu") -> torch.Tensor:
+    g = _gen(device, seed)
+    if kind == "gauss1":
+        y = _randn((M, N), g, device)
+    elif kind == "gauss_1e-4":
+        y = _randn((M, N), g, device) * 1e-4
+    elif kind == "lognormal_rows":
+        y = _randn((M, N), g, device) * 1e-4
+        z = _randn((M, 1), g, device)
+        y = y * torch.exp(z)
+    else:
+        raise ValueError(kind)
+    return y.to(torch.bfloat16)
+
+
+def linear_inputs(cfg: str, seed: int = 0, device="cpu"):
+    """(X [M,K], W [N,K], dY [M,N]) bf16 for a named linear-layer workload."""
+    M, K, N = SHAPES[cfg]
+    if cfg == "tiny":
+        x = make_x(M, K, "gauss", seed, device)
+        w = make_w(N, K, seed + 1, std=0.02, device=device)
+        dy = make_dy(M, N, "gauss1", seed + 2, device)
+    elif cfg == "llm1p9b":
+        x = make_x(M, K, "t3_outlier_channels", seed, device)
+        w = make_w(N, K, seed + 1, device=device)
+        dy = make_dy(M, N, "gauss_1e-4", seed + 2, device)
+    elif cfg == "mlp8b_up":
+        x = make_x(M, K, "gauss", seed, device)
+        w = make_w(N, K, seed + 1, device=device)
+        dy = make_dy(M, N, "lognormal_rows", seed + 2, device)
+    elif cfg == "mlp8b_down":
+        x = make_x(M, K, "silu_gated", seed, device)
+        w = make_w(N, K, seed + 1, device=device)
+        dy = make_dy(M, N, "lognormal_rows", seed + 2, device)
+    else:
+        raise ValueError(cfg)
+    return x, w, dy
+
+
+def custom_linear_inputs(M: int, K: int, N: int, seed: int = 0, device="cpu", x_kind="t3_outlier_channels",
+                         dy_kind="lognormal_rows"):
+    """Inputs of an arbitrary shape with the llm1p9b-style distributions (used for ragged and
+    multi-tile parity cases)."""
+    return (make_x(M, K, x_kind, seed, device), make_w(N, K, seed + 1, device=device),
+            make_dy(M, N, dy_kind, seed + 2, device))
+
+
+def sweep_tensor(numel_log2: int, L: int, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Quantizer-sweep input: 2^p elements as rows of length L (rows rounded to a multiple of
+    128, at least 128), N(0,1) with 0.1% of elements x50."""
+    rows = max(128, int(round((2 ** numel_log2) / L / 128.0)) * 128)
+    g = _gen(device, seed)
+    x = _randn((rows, L), g, device)
+    mask = torch.rand((rows, L), generator=g, device=device) < 1e-3
+    x = torch.where(mask, x * 50.0, x)
+    return x.to(torch.bfloat16)
+
+
+def sweep_rows(numel_log2: int, L: int) -> int:
+    return max(128, int(round((2 ** numel_log2) / L / 128.0)) * 128)
+

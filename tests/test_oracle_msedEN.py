@@ -1,0 +1,206 @@
+"""Pins of the oracle's MS-EDEN quantizer (CPU only).
+
+Independent checks: codes against library RNE of the rotated values (with the rotation
+itself pinned to the dense Hadamard in test_oracle_rotation); the EDEN identity
+<S Q(y), y> = <y, y>; scales that are a valid stochastic rounding of S*p/g, RNE below the
+2^-6 cutoff; unbiasedness of the dequantized estimate over 4096 seeds; the MSE ratio to the
+elementwise-SR baseline ("more than 2x lower error").
+"""
+import ml_dtypes
+import numpy as np
+import torch
+
+import oracle as O
+
+
+def _bf16(a) -> torch.Tensor:
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def _unpack(codes: np.ndarray) -> np.ndarray:
+    out = np.empty((codes.shape[0], codes.shape[1] * 2), np.uint8)
+    out[:, 0::2] = codes & 15
+    out[:, 1::2] = codes >> 4
+    return out
+
+
+def _rotated(xb: torch.Tensor, seed: int) -> np.ndarray:
+    """fp32 rotated rows, via the pinned butterfly."""
+    xf = xb.float().numpy()
+    sgn = O.rht_signs(seed)
+    R, C = xf.shape
+    y = np.empty_like(xf)
+    for r in range(R):
+        for b in range(C // 128):
+            y[r, 128 * b:128 * b + 128] = O.fwht128((sgn * xf[r, 128 * b:128 * b + 128]).astype(np.float32))
+    return y
+
+
+def _inputs(seed=0, R=16, C=512):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((R, C)).astype(np.float32) * 1e-2
+    x[1] *= 1e-4
+    x[2, :128] = 0.0
+    x[3, 5] = 3.0
+    x[4] *= np.exp(rng.standard_normal(C)).astype(np.float32)
+    return _bf16(x)
+
+
+def test_codes_are_library_rne_of_rotated_values():
+    x = _inputs()
+    seed = 11
+    v = O.msedEN(x, seed, 1, "row")
+    y = _rotated(x, seed)
+    codes = _unpack(v.codes)
+    R, C = y.shape
+    for r in range(R):
+        for q in range(C // 16):
+            yq = y[r, 16 * q:16 * q + 16]
+            a = np.float32(np.max(np.abs(yq)))
+            assert v.amax_g[r, q] == a
+            if a < 2.0 ** -100:
+                assert np.array_equal(codes[r, 16 * q:16 * q + 16], np.where(np.signbit(yq), 8, 0))
+                continue
+            p = np.float32(a / np.float32(6.0))
+            rc = np.float32(np.float32(1.0) / p)
+            lib = (yq * rc).astype(np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 15
+            assert np.array_equal(codes[r, 16 * q:16 * q + 16], lib)
+
+
+def test_eden_identity_and_prescale():
+    """S makes the corrected estimate S*Q(y) have the same projection on y as y itself."""
+    x = _inputs(1)
+    v = O.msedEN(x, 5, 1, "row")
+    y = _rotated(x, 5).astype(np.float64)
+    codes = _unpack(v.codes)
+    val = np.array([O.e2m1_value(c) for c in range(16)])[codes]
+    p = (v.amax_g.astype(np.float32) / np.float32(6.0)).astype(np.float64)
+    p[v.amax_g < 2.0 ** -100] = 0.0
+    Q = val * np.repeat(p, 16, axis=1)
+    R, C = y.shape
+    for r in range(R):
+        for b in range(C // 128):
+            sl = slice(128 * b, 128 * b + 128)
+            yy = y[r, sl] @ y[r, sl]
+            qy = Q[r, sl] @ y[r, sl]
+            S = float(v.S[r, b])
+            if qy > 0:
+                assert abs(S * qy - yy) <= 1e-5 * yy
+            else:
+                assert S == 1.0
+            for q in range(8):
+                gi = 8 * b + q
+                assert v.P[r, gi] == np.float32(np.float32(S) * np.float32(p[r, gi]))
+
+
+def test_scales_are_valid_sr_and_rne_below_cutoff():
+    x = _inputs(2)
+    v = O.msedEN(x, 9, 2, "row")
+    ginv = np.float32(np.float32(1.0) / v.g)
+    vals = np.array([O.e4m3_value(c) for c in range(127)])
+    n_sr = n_rne = 0
+    for j, (P, s) in enumerate(zip(v.P.ravel(), v.scales.ravel())):
+        t = float(np.float32(P * ginv))
+        if t < 2.0 ** -6:
+            assert s == O.e4m3_rne(t)     # RNE below the E4M3 normal range
+            n_rne += 1
+        else:
+            lo = vals[vals <= t].max()
+            hi = vals[vals >= t].min()
+            assert O.e4m3_value(s) in (lo, hi)
+            n_sr += 1
+    assert n_sr > 100 and n_rne > 0
+    assert v.g == np.float32(np.float32(v.amax) / np.float32(1536.0))
+
+
+def test_col_view_is_row_view_of_transpose():
+    x = _inputs(3, R=256, C=128)
+    a = O.msedEN(x, 4, 3, "col")
+    b = O.msedEN(x.t().contiguous(), 4, 3, "row")
+    assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales, b.scales) and a.g == b.g
+
+
+def _estimate(x, seed, tid=1):
+    v = O.msedEN(x, seed, tid, "row")
+    return O.unrotate(v.dequant(), seed)
+
+
+def _mean_stats(fn, xd, B):
+    s1 = np.zeros_like(xd)
+    s2 = np.zeros_like(xd)
+    for seed in range(B):
+        e = fn(1000 + seed)
+        s1 += e
+        s2 += e * e
+    mean = s1 / B
+    var = np.maximum(s2 / B - mean ** 2, 1e-300)
+    z = (mean - xd) / np.sqrt(var / B)
+    rel_bias = np.linalg.norm(mean - xd) / np.linalg.norm(xd)
+    rel_noise = np.sqrt(var.mean()) / np.sqrt((xd ** 2).mean())
+    return z, rel_bias, rel_noise
+
+
+def test_unbiased_over_4096_seeds():
+    """Mean of the dequantized MS-EDEN estimate over 4096 seeds converges to x: the bias of
+    almost every coordinate is below 3 standard errors of the 4096-sample mean.
+
+    A fixed 128-point randomized Hadamard rotation is a compromise the pages name ("Question 1":
+    fixed 128-dim rotation groups, shared rotation); EDEN is exactly unbiased only for a
+    uniformly random rotation, and with the Hadamard a residual bias of about 2% of the
+    per-sample error remains, visible at B = 4096 in a few coordinates.  So the check is
+    aggregate: <= 3% of coordinates beyond 3 SE (0.27% expected without any bias) and a
+    relative bias below 5% of the relative per-sample error."""
+    rng = np.random.default_rng(7)
+    xf = rng.standard_normal((2, 256)).astype(np.float32)
+    xf[0, 17] = 9.0
+    x = _bf16(xf)
+    xd = x.float().numpy().astype(np.float64)
+    z, rel_bias, rel_noise = _mean_stats(lambda s: _estimate(x, s), xd, 4096)
+    assert np.mean(np.abs(z) > 3) <= 0.03, np.mean(np.abs(z) > 3)
+    assert rel_bias < 0.05 * rel_noise, (rel_bias, rel_noise)
+    # Control: RTN on the rotated values without the EDEN factor and with exact scales is
+    # biased -- its mean stays far from x.
+    def rtn_no_eden(seed):
+        v = O.msedEN(x, seed, 1, "row")
+        p = (v.amax_g / np.float32(6.0)).astype(np.float64)
+        val = np.array([O.e2m1_value(c) for c in range(16)])[_unpack(v.codes)]
+        return O.unrotate(val * np.repeat(p, 16, axis=1), seed)
+    zb, rel_bias_rtn, _ = _mean_stats(rtn_no_eden, xd, 1024)
+    assert rel_bias_rtn > 2 * rel_bias
+    # Control: the forward quantizer (RTN + 4/6, no rotation) is deterministic, so its
+    # "mean" is its own quantization error, an order of magnitude above MS-EDEN's bias.
+    v46 = O.fwd46(x)
+    assert np.linalg.norm(v46.dequant() - xd) / np.linalg.norm(xd) > 10 * rel_bias
+
+
+def test_sr_baseline_unbiased():
+    rng = np.random.default_rng(9)
+    x = _bf16(rng.standard_normal((2, 256)))
+    xd = x.float().numpy().astype(np.float64)
+    z, rel_bias, rel_noise = _mean_stats(lambda s: O.unrotate(O.sr_dequant(x, s, 7, "row"), s), xd, 2048)
+    assert np.mean(np.abs(z) > 3) <= 0.03 and rel_bias < 0.05 * rel_noise
+
+
+def test_mse_ratio_to_sr():
+    """MSE(SR) / MSE(MS-EDEN) on Gaussian data.  The pages report more than 2x lower error for
+    MS-EDEN.  Measured here: about 2.2 against unbiased NVFP4 SR (group scale rounded up so no
+    element clips); 1.85 against SR with round-to-nearest scales, which clip and are slightly
+    biased.  Require >= 1.8 (finite-sample margin)."""
+    rng = np.random.default_rng(8)
+    x = _bf16(rng.standard_normal((64, 1024)))
+    mse_e = mse_s = 0.0
+    for seed in range(4):
+        v = O.msedEN(x, seed, 1, "row")
+        y = _rotated(x, seed).astype(np.float64)
+        mse_e += np.mean((v.dequant() - y) ** 2)
+        mse_s += np.mean((O.sr_dequant(x, seed, 7, "row") - y) ** 2)
+    ratio = mse_s / mse_e
+    assert ratio >= 1.8, ratio
+
+
+def test_flushed_and_zero_views():
+    z = O.msedEN(_bf16(np.zeros((4, 128))), 0, 1, "row")
+    assert z.g == 1.0 and np.all(z.scales == 0) and np.all(z.S == 1.0)
+    tiny = _bf16(np.full((4, 128), 1e-33, np.float32))
+    t = O.msedEN(tiny, 0, 1, "row")
+    assert np.all(t.amax_g < 2.0 ** -100) and np.all(t.scales == 0) and t.g == 1.0
