@@ -1,0 +1,163 @@
+/*
+ * qt2.h -- C ABI of the Quartet II NVFP4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * Citations (page title, then section):
+ *   [QII-th] "Quartet II ... MS-EDEN" Thai translation (itsolotime.com archives 22992): abstract,
+ *            "Question 1" (fixed 128-dim rotation groups, shared rotation, small FP8 scales), §1.
+ *   [QII-ru] Quartet II review, D. Avetisyan (denisavetisyan.com ?p=3427): "NVFP4 and
+ *            micro-scaling", "Unbiased quantization with MS-EDEN and randomized methods".
+ *   [FAF]    "Format-Aware Fusion for Fast FP4 Pretraining" (rit.work blog): "the speed-up is lost
+ *            between the matmuls" (global scale sync point; both layouts from one producer).
+ *   [QII-tg] Quartet II digest (quant_prune_distill post 640): "Method".
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device; the caller owns all
+ *     memory (inputs, outputs, workspace).  Nothing is allocated by the library.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Returning QT2_OK means the launches were enqueued, not that they finished.
+ *   - Arguments are validated on the host before any launch; on error nothing is enqueued and
+ *     a negative qt2_status is returned.  Launch failures map to QT2_ERR_CUDA.  No call aborts.
+ *   - bf16 matrices are row-major with a leading dimension `ld` (elements between rows,
+ *     ld >= cols, ld a multiple of 8) and 16-byte aligned base pointers.
+ *   - Every dimension must be a positive multiple of 128.
+ *   - The device must be compute capability 10.0 (B200); otherwise QT2_ERR_DEVICE.
+ *
+ * NVFP4 view layout (one quantized operand of a "TN" GEMM, grouped along its contraction axis):
+ *   R = rows (non-contraction axis), C = columns (contraction axis), both multiples of 128.
+ *   codes        [R][C/2] bytes, row-major; element 2j in the low nibble of byte j, element 2j+1
+ *                in the high nibble.  Nibble = E2M1: bit 3 sign, bits 2..0 index into
+ *                {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   scales       one unsigned E4M3 byte per 16-element group, R*C/16 bytes, in the tensor-core
+ *                scale-factor order: the scale of row r, group j (0 <= j < C/16) is at byte
+ *                  ((r/128)*(C/64) + j/4)*512 + (r%32)*16 + ((r%128)/32)*4 + (j%4).
+ *   tensor_scale one fp32 g.  The value of element (r, c) is  val(code) * E4M3(scale) * g.
+ */
+#ifndef QT2_H
+#define QT2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QT2_API __attribute__((visibility("default")))
+#else
+#define QT2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qt2_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+    QT2_OK = 0,
+    QT2_ERR_INVALID_ARG = -1, /* null pointer, bad enum, unsupported layout request */
+    QT2_ERR_SHAPE = -2,       /* a dimension not a positive multiple of 128, or ld < cols */
+    QT2_ERR_ALIGN = -3,       /* a pointer not 16-byte aligned, or ld not a multiple of 8 */
+    QT2_ERR_WORKSPACE = -4,   /* workspace null or smaller than the size query returned */
+    QT2_ERR_CUDA = -5,        /* a CUDA runtime/driver call or launch failed */
+    QT2_ERR_TIMEOUT = -6,     /* a device-side bounded wait gave up (see qt2_device_status) */
+    QT2_ERR_DEVICE = -7       /* no device, or the current device is not sm_100 */
+} qt2_status;
+
+enum { QT2_LAYOUT_ROW = 1, QT2_LAYOUT_COL = 2, QT2_LAYOUT_BOTH = 3 };
+enum { QT2_DTYPE_BF16 = 0, QT2_DTYPE_F32 = 1 };
+
+/* Tensor ids of the Philox streams used by qt2_linear_bwd (id 0 draws the rotation signs). */
+enum { QT2_TID_SIGNS = 0, QT2_TID_DY_ROW = 1, QT2_TID_DY_COL = 2, QT2_TID_W_COL = 3, QT2_TID_X_COL = 4 };
+
+typedef struct {
+    void *codes;         /* device, R*C/2 bytes */
+    void *scales;        /* device, R*C/16 bytes, scale-factor order above */
+    float *tensor_scale; /* device, 1 float */
+} qt2_nvfp4_view;
+
+QT2_API int qt2_version(void);
+QT2_API const char *qt2_status_string(qt2_status s);
+
+/* Reads and clears the library's device-side status word after synchronizing `stream`.
+ * *code = 0 when no kernel reported a problem; QT2_ERR_TIMEOUT when a bounded wait gave up.
+ * Synchronizes the stream; meant for tests and debugging, not the hot path. */
+QT2_API qt2_status qt2_device_status(qt2_stream_t stream, int *code);
+
+/* ---------------------------------------------------------------------------------------
+ * Forward quantizer: round-to-nearest onto E2M1 in 1x16 groups with the "4/6" grid choice.
+ * [QII-tg] "Method": per group the full grid (+-6) or the truncated grid (+-4) is used,
+ * whichever gives the smaller quantization error; 1x16 groups rather than 16x16 blocks.
+ * [QII-th] "fairness" answer: the forward pass uses RTN.  [FAF]: the fp32 tensor scale depends
+ * on the tensor-wide max, a sync point before packing.
+ *
+ * x_bf16 [rows][cols] (leading dimension ld) is grouped along cols.  Computes A = max|x|,
+ * g = A/1792 (g = 1 and an all-zero result when A < 2^-100), then per group, for k = 6 then 4:
+ * s_k = RNE_E4M3(a/(g*k)), d = s_k*g, codes = RNE_E2M1(x * (1/d)), err_k = sum (x - val*d)^2;
+ * keeps k = 4 iff err_4 < err_6.  Results are bit-identical to the reference algorithm.
+ * layout_mask must be QT2_LAYOUT_ROW (the forward GEMM consumes row views only); row_out
+ * receives the view (R = rows, C = cols); col_out is ignored and may be NULL.
+ * Workspace: at least qt2_quant_fwd46_workspace_size() bytes, 16-byte aligned; it holds the
+ * tensor max and is overwritten.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_fwd46_workspace_size(int64_t rows, int64_t cols, size_t *bytes);
+QT2_API qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                           const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                           size_t ws_bytes, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Backward quantizer MS-EDEN (MicroScaling EDEN).  [QII-tg] "Method": a random Hadamard rotation
+ * and a factor <x,x>/<Q(Rx),Rx> (EDEN), plus stochastic rounding of the FP8 scales;
+ * [QII-th] "Question 1": fixed 128-element rotation groups, one shared rotation and seed, and
+ * no SR for very small scales.  [FAF]: one producer emits both layouts the backward GEMMs need.
+ *
+ * x_bf16 [rows][cols] (leading dimension ld).  A view groups along the contraction axis:
+ *   QT2_LAYOUT_ROW: groups along cols -> row_out view with R = rows, C = cols
+ *   QT2_LAYOUT_COL: groups along rows -> col_out view of x^T with R = cols, C = rows
+ *   QT2_LAYOUT_BOTH: both views from one read of x.
+ * Per 128-block of the grouped axis: y = H D x (D = the 128 signs of Philox(seed, tensor id 0),
+ * bit i of word i/32 set -> -1; H = unnormalised Sylvester Hadamard, butterfly strides 1..64);
+ * per group p = max|y|/6, codes = RNE_E2M1(y * (1/p)); per block S = sum y^2 / sum p*<val, y>;
+ * view tensor scale g = max|y|/1536; group scale = SR_E4M3(S*p/g) with the draw of canonical
+ * group index r*(C/16)+j from Philox(seed, tensor_id of the view), RNE below 2^-6.
+ * The rotated views multiply with alpha = 2^-7 (qt2_gemm_nvfp4).  Bit-identical to the
+ * reference algorithm for the same seed and tensor ids.
+ * Workspace: at least qt2_quant_msedEN_workspace_size() bytes, 256-byte aligned (pre-scales
+ * S*p in fp32 and the view maxima); overwritten.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_msedEN_workspace_size(int64_t rows, int64_t cols, int layout_mask, size_t *bytes);
+QT2_API qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                            uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
+                            const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                            size_t ws_bytes, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Block-scaled NVFP4 GEMM on the 5th-generation tensor cores ([QII-th] abstract and §1: NVFP4 is
+ * natively supported by Blackwell GPUs).  "TN": a is an [M][K] view, b an [N][K] view, both
+ * grouped along K.  c[m][n] = alpha * gA * gB * sum_k val(a)*sa * val(b)*sb, accumulated in fp32,
+ * written as bf16 or fp32 (c_dtype) with leading dimension ldc >= N (a multiple of 8).
+ * alpha = 1 for forward operands, 2^-7 for two MS-EDEN operands sharing a rotation.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_gemm_nvfp4(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,
+                          float alpha, void *c, int c_dtype, int64_t ldc, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Quartet II linear layer ([QII-ru] "Unbiased quantization ...": a computation graph with every
+ * linear-layer GEMM in NVFP4; [QII-th] abstract: better estimates in all major matmuls).
+ * x [M][K], w [N][K] (PyTorch Linear layout), dy [M][N]; all bf16, contiguous.
+ * Forward:  y = X W^T with both operands through the forward quantizer; y bf16 [M][N].
+ * Backward: dX = dY W  (dY row view, W column view, rotated along N),
+ *           dW = dY^T X (dY column view, X column view, rotated along M),
+ *           tensor ids QT2_TID_*; dx bf16 [M][K]; dw [N][K] bf16 or fp32 (dw_dtype).
+ * Workspace: the size queries below; 256-byte aligned; holds the quantized views.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes);
+QT2_API qt2_status qt2_linear_fwd(const void *x, const void *w, int64_t M, int64_t K, int64_t N, void *y_bf16,
+                          void *workspace, size_t ws_bytes, qt2_stream_t stream);
+QT2_API qt2_status qt2_linear_bwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes);
+QT2_API qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t M, int64_t K, int64_t N,
+                          uint64_t seed, void *dx_bf16, void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
+                          qt2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QT2_H */

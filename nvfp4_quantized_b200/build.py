@@ -1,0 +1,58 @@
+"""Build the qt2 CUDA library in-tree: nvfp4_quantized_b200/libqt2.so (sm_100a only).
+
+    python -m nvfp4_quantized_b200.build [--force] [--verbose]
+
+nvcc cross-compiles without a GPU.  --fmad=false keeps every floating-point expression of
+the quantizers an individually rounded IEEE operation (they also use explicit _rn intrinsics).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libqt2.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
+                  glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "qt2.h")])
+
+
+def nvcc_cmd(out: str, verbose: bool = False):
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "--fmad=false", "-std=c++17",
+           "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared", "-I", INCLUDE, "-I", CSRC,
+           "-o", out, os.path.join(CSRC, "qt2_lib.cu")]
+    if verbose:
+        cmd[1:1] = ["-Xptxas", "-v"]
+    return cmd
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    newest = max(os.path.getmtime(p) for p in sources())
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not verbose:
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    res = subprocess.run(nvcc_cmd(tmp, verbose), capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libqt2.so")
+    if verbose:
+        sys.stderr.write(res.stdout + res.stderr)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    a = ap.parse_args()
+    print(build(a.force, a.verbose))

@@ -1,0 +1,44 @@
+// qt2_internal.h -- declarations shared by the qt2 library's translation units (host side).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "qt2.h"
+
+namespace qt2 {
+
+// One quantized view on the device (see the layout in qt2.h).
+struct DevView {
+    uint8_t *codes;
+    uint8_t *scales;
+    float *tensor_scale;
+};
+
+// Tensor-scale constants and the flush threshold of the quantizers.
+constexpr float kFwd46Denominator = 1792.0f;   // 4 * 448: both 4/6 candidates keep scales <= 448
+constexpr float kMsedDenominator = 1536.0f;    // 6 * 256: 1.75x headroom for the EDEN factor and SR
+constexpr float kTiny = 0x1p-100f;             // below this a tensor (fwd46) or a group (MS-EDEN) is zero
+constexpr float kSrCutoff = 0x1p-6f;           // E4M3 scales below 2^-6 are rounded to nearest
+
+// Kernel launchers (one translation unit: qt2_lib.cu).  Each returns the launch status.
+cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *amax_word,
+                             cudaStream_t s);
+cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
+                              DevView out, cudaStream_t s);
+cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col,
+                              uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
+                              uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s);
+cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
+                                 uint32_t tid, DevView out, cudaStream_t s);
+cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
+                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s);
+
+// 2D tensor map for TMA (no multicast anywhere in this library).
+bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+}  // namespace qt2

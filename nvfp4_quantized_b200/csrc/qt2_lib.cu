@@ -1,0 +1,480 @@
+// qt2_lib.cu -- the qt2 library: kernel launchers and the C ABI declared in include/qt2.h.
+//
+// One translation unit (the kernels are included) so that the device status word is a single
+// symbol.  Built for sm_100a only:
+//   nvcc -gencode arch=compute_100a,code=sm_100a -O3 -lineinfo --fmad=false -shared ...
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "qt2_internal.h"
+#include "qt2_device.cuh"
+#include "quant_kernels.cuh"
+#include "gemm_kernel.cuh"
+
+namespace qt2 {
+
+// ---------------------------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------------------------
+static int sm_count() {
+    static std::atomic<int> cached{0};
+    int v = cached.load();
+    if (v == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        if (v <= 0) v = 148;
+        cached.store(v);
+    }
+    return v;
+}
+
+cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *amax_word,
+                             cudaStream_t s) {
+    const int64_t warps_needed = R;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps_needed + 7) / 8, (int64_t)sm_count() * 8));
+    amax_bf16_kernel<<<blocks, 256, 0, s>>>(x, R, C, ld, amax_word);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
+                              DevView out, cudaStream_t s) {
+    const int64_t groups = R * (C >> 4);
+    const int64_t blocks = std::min<int64_t>((groups + 255) / 256, (int64_t)sm_count() * 64);
+    fwd46_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, R, C, ld, amax_word, out.codes, out.scales,
+                                                       out.tensor_scale);
+    return cudaGetLastError();
+}
+
+static constexpr int kMsedSmem = 32768 + 1024;
+
+template <bool ROW, bool COL>
+static cudaError_t launch_msed_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed, DevView row,
+                                       DevView col, float *P_row, float *P_col, uint32_t *amax_row,
+                                       uint32_t *amax_col, cudaStream_t s) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(msed_tile_kernel<ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kMsedSmem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    dim3 grid((unsigned)(C / 128), (unsigned)(R / 128));
+    msed_tile_kernel<ROW, COL><<<grid, 128, kMsedSmem, s>>>(tmap, R, C, seed, row.codes, P_row, amax_row, col.codes,
+                                                             P_col, amax_col);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col,
+                              uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
+                              uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s) {
+    if (do_row && do_col)
+        return launch_msed_variant<true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+    if (do_row)
+        return launch_msed_variant<true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+    return launch_msed_variant<false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+}
+
+cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
+                                 uint32_t tid, DevView out, cudaStream_t s) {
+    const int64_t words = (R * C) >> 6;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((words + 255) / 256, (int64_t)sm_count() * 16));
+    msed_finalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(P), R, C, amax_word, seed,
+                                                          tid, reinterpret_cast<uint32_t *>(out.scales),
+                                                          out.tensor_scale);
+    return cudaGetLastError();
+}
+
+template <int BN>
+static cudaError_t launch_gemm_bn(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
+                                  int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
+                                  cudaStream_t s) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        GemmCfg<BN>::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    dim3 grid((unsigned)(N / BN), (unsigned)(M / kGemmBM));
+    gemm_nvfp4_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, s>>>(
+        tmA, tmB, a.scales, b.scales, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)K, c_dtype);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
+                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s) {
+    if (N % 256 == 0) return launch_gemm_bn<256>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
+    return launch_gemm_bn<128>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime; no libcuda link needed)
+// ---------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace qt2
+
+// =============================================================================================
+// C ABI
+// =============================================================================================
+using namespace qt2;
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dim_ok(int64_t d) { return d > 0 && d % 128 == 0 && d <= (int64_t(1) << 31); }
+
+qt2_status check_device() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return QT2_ERR_DEVICE;
+    }
+    if (dev < 64) {
+        int v = cached[dev].load();
+        if (v == 1) return QT2_OK;
+        if (v == 2) return QT2_ERR_DEVICE;
+    }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QT2_ERR_DEVICE;
+    }
+    const bool ok = (major == 10 && minor == 0);
+    if (dev < 64) cached[dev].store(ok ? 1 : 2);
+    return ok ? QT2_OK : QT2_ERR_DEVICE;
+}
+
+qt2_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QT2_OK : QT2_ERR_CUDA; }
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+    uint8_t *base;
+    size_t used = 0;
+    explicit Carve(void *b) : base(static_cast<uint8_t *>(b)) {}
+    uint8_t *take(size_t bytes) {
+        uint8_t *p = base ? base + used : nullptr;
+        used = align_up(used + bytes, kWsAlign);
+        return p;
+    }
+};
+
+bool view_ok(const qt2_nvfp4_view *v) {
+    return v && v->codes && v->scales && v->tensor_scale && aligned16(v->codes) && aligned16(v->scales) &&
+           (reinterpret_cast<uintptr_t>(v->tensor_scale) & 3u) == 0;
+}
+
+DevView dev_view(const qt2_nvfp4_view *v) {
+    return DevView{static_cast<uint8_t *>(v->codes), static_cast<uint8_t *>(v->scales), v->tensor_scale};
+}
+
+// Workspace of one MS-EDEN call: amax words (2), then P_row, P_col.
+size_t msed_ws(int64_t rows, int64_t cols, int mask, float **P_row, float **P_col, uint32_t **amax, void *ws) {
+    Carve c(ws);
+    *amax = reinterpret_cast<uint32_t *>(c.take(2 * sizeof(uint32_t)));
+    *P_row = (mask & QT2_LAYOUT_ROW) ? reinterpret_cast<float *>(c.take((size_t)rows * cols / 16 * 4)) : nullptr;
+    *P_col = (mask & QT2_LAYOUT_COL) ? reinterpret_cast<float *>(c.take((size_t)rows * cols / 16 * 4)) : nullptr;
+    return c.used;
+}
+
+qt2_status validate_bf16(const void *x, int64_t rows, int64_t cols, int64_t ld) {
+    if (!x) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols) || ld < cols) return QT2_ERR_SHAPE;
+    if (!aligned16(x) || ld % 8 != 0) return QT2_ERR_ALIGN;
+    return QT2_OK;
+}
+
+// Enqueue an MS-EDEN quantization of x (rows x cols, ld) into the requested views.
+qt2_status msed_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, int mask, uint64_t seed, uint32_t tid_row,
+                        uint32_t tid_col, DevView row, DevView col, float *P_row, float *P_col, uint32_t *amax,
+                        cudaStream_t s) {
+    CUtensorMap tmap;
+    if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
+                        128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return QT2_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_msed_tiles(tmap, rows, cols, (mask & QT2_LAYOUT_ROW) != 0, (mask & QT2_LAYOUT_COL) != 0, seed, row, col,
+                          P_row, P_col, amax, amax + 1, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    if (mask & QT2_LAYOUT_ROW) {
+        e = launch_msed_finalize(P_row, rows, cols, amax, seed, tid_row, row, s);
+        if (e != cudaSuccess) return QT2_ERR_CUDA;
+    }
+    if (mask & QT2_LAYOUT_COL) {
+        e = launch_msed_finalize(P_col, cols, rows, amax + 1, seed, tid_col, col, s);
+        if (e != cudaSuccess) return QT2_ERR_CUDA;
+    }
+    return QT2_OK;
+}
+
+qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *amax,
+                         cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_fwd46_rows(static_cast<const uint16_t *>(x), rows, cols, ld, amax, out, s);
+    return from_cuda(e);
+}
+
+qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, float alpha, void *c, int c_dtype,
+                        int64_t ldc, cudaStream_t s) {
+    CUtensorMap tmA, tmB;
+    const int bn = (N % 256 == 0) ? 256 : 128;
+    if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
+                        kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b.codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
+                        (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B))
+        return QT2_ERR_CUDA;
+    return from_cuda(launch_gemm_nvfp4(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
+}
+
+// Views carved from a workspace: codes, scales, tensor scale.
+DevView carve_view(Carve &c, int64_t R, int64_t C) {
+    DevView v;
+    v.codes = c.take((size_t)R * C / 2);
+    v.scales = c.take((size_t)R * C / 16);
+    v.tensor_scale = reinterpret_cast<float *>(c.take(sizeof(float)));
+    return v;
+}
+
+size_t linear_fwd_layout(int64_t M, int64_t K, int64_t N, void *ws, DevView *vx, DevView *vw, uint32_t **amax) {
+    Carve c(ws);
+    *amax = reinterpret_cast<uint32_t *>(c.take(2 * sizeof(uint32_t)));
+    *vx = carve_view(c, M, K);
+    *vw = carve_view(c, N, K);
+    return c.used;
+}
+
+struct BwdLayout {
+    DevView dy_row, dy_col, w_col, x_col;
+    float *P_dy_row, *P_dy_col, *P_w_col, *P_x_col;
+    uint32_t *amax;   // 6 words: dY row/col, W (col at +1), X (col at +1)
+};
+
+size_t linear_bwd_layout(int64_t M, int64_t K, int64_t N, void *ws, BwdLayout *L) {
+    Carve c(ws);
+    L->amax = reinterpret_cast<uint32_t *>(c.take(6 * sizeof(uint32_t)));
+    L->dy_row = carve_view(c, M, N);
+    L->dy_col = carve_view(c, N, M);
+    L->w_col = carve_view(c, K, N);
+    L->x_col = carve_view(c, K, M);
+    L->P_dy_row = reinterpret_cast<float *>(c.take((size_t)M * N / 16 * 4));
+    L->P_dy_col = reinterpret_cast<float *>(c.take((size_t)M * N / 16 * 4));
+    L->P_w_col = reinterpret_cast<float *>(c.take((size_t)N * K / 16 * 4));
+    L->P_x_col = reinterpret_cast<float *>(c.take((size_t)M * K / 16 * 4));
+    return c.used;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qt2_version(void) { return 100; }
+
+const char *qt2_status_string(qt2_status s) {
+    switch (s) {
+        case QT2_OK: return "ok";
+        case QT2_ERR_INVALID_ARG: return "invalid argument";
+        case QT2_ERR_SHAPE: return "bad shape (dimensions must be positive multiples of 128, ld >= cols)";
+        case QT2_ERR_ALIGN: return "misaligned pointer or leading dimension (16-byte alignment required)";
+        case QT2_ERR_WORKSPACE: return "workspace missing or too small";
+        case QT2_ERR_CUDA: return "CUDA error";
+        case QT2_ERR_TIMEOUT: return "device-side wait timed out";
+        case QT2_ERR_DEVICE: return "no sm_100 device";
+    }
+    return "unknown status";
+}
+
+qt2_status qt2_device_status(qt2_stream_t stream, int *code) {
+    if (!code) return QT2_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QT2_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return QT2_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return QT2_ERR_CUDA;
+    *code = v;
+    return QT2_OK;
+}
+
+qt2_status qt2_quant_fwd46_workspace_size(int64_t rows, int64_t cols, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols)) return QT2_ERR_SHAPE;
+    *bytes = kWsAlign;
+    return QT2_OK;
+}
+
+qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                           const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                           size_t ws_bytes, qt2_stream_t stream) {
+    (void)col_out;
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (layout_mask != QT2_LAYOUT_ROW || !row_out) return QT2_ERR_INVALID_ARG;
+    if (!view_ok(row_out)) return row_out->codes && row_out->scales && row_out->tensor_scale ? QT2_ERR_ALIGN
+                                                                                             : QT2_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < kWsAlign) return QT2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QT2_ERR_ALIGN;
+    if ((st = check_device()) != QT2_OK) return st;
+    return fwd46_enqueue(x_bf16, rows, cols, ld, dev_view(row_out), static_cast<uint32_t *>(workspace),
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+qt2_status qt2_quant_msedEN_workspace_size(int64_t rows, int64_t cols, int layout_mask, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols)) return QT2_ERR_SHAPE;
+    float *a, *b;
+    uint32_t *c;
+    *bytes = msed_ws(rows, cols, layout_mask, &a, &b, &c, nullptr);
+    return QT2_OK;
+}
+
+qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                            uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
+                            const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                            size_t ws_bytes, qt2_stream_t stream) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_ROW) && !view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_COL) && !view_ok(col_out)) return col_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    float *P_row, *P_col;
+    uint32_t *amax;
+    if (ws_bytes < msed_ws(rows, cols, layout_mask, &P_row, &P_col, &amax, workspace)) return QT2_ERR_WORKSPACE;
+    if ((st = check_device()) != QT2_OK) return st;
+    const DevView none{nullptr, nullptr, nullptr};
+    return msed_enqueue(x_bf16, rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
+                        (layout_mask & QT2_LAYOUT_ROW) ? dev_view(row_out) : none,
+                        (layout_mask & QT2_LAYOUT_COL) ? dev_view(col_out) : none, P_row, P_col, amax,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+qt2_status qt2_gemm_nvfp4(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,
+                          float alpha, void *c, int c_dtype, int64_t ldc, qt2_stream_t stream) {
+    if (!a || !b || !c) return QT2_ERR_INVALID_ARG;
+    if (c_dtype != QT2_DTYPE_BF16 && c_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K) || ldc < N) return QT2_ERR_SHAPE;
+    if (!view_ok(a) || !view_ok(b)) return (a->codes && a->scales && a->tensor_scale && b->codes && b->scales &&
+                                            b->tensor_scale)
+                                               ? QT2_ERR_ALIGN
+                                               : QT2_ERR_INVALID_ARG;
+    if (!aligned16(c) || ldc % 8 != 0) return QT2_ERR_ALIGN;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    return gemm_enqueue(dev_view(a), dev_view(b), M, N, K, alpha, c, c_dtype, ldc,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+qt2_status qt2_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    DevView a, b;
+    uint32_t *w;
+    *bytes = linear_fwd_layout(M, K, N, nullptr, &a, &b, &w);
+    return QT2_OK;
+}
+
+qt2_status qt2_linear_fwd(const void *x, const void *w, int64_t M, int64_t K, int64_t N, void *y_bf16,
+                          void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    if (!x || !w || !y_bf16) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y_bf16)) return QT2_ERR_ALIGN;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    DevView vx, vw;
+    uint32_t *amax;
+    if (ws_bytes < linear_fwd_layout(M, K, N, workspace, &vx, &vw, &amax)) return QT2_ERR_WORKSPACE;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = fwd46_enqueue(x, M, K, K, vx, amax, s)) != QT2_OK) return st;
+    if ((st = fwd46_enqueue(w, N, K, K, vw, amax + 1, s)) != QT2_OK) return st;
+    return gemm_enqueue(vx, vw, M, N, K, 1.0f, y_bf16, QT2_DTYPE_BF16, N, s);
+}
+
+qt2_status qt2_linear_bwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    BwdLayout L;
+    *bytes = linear_bwd_layout(M, K, N, nullptr, &L);
+    return QT2_OK;
+}
+
+qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t M, int64_t K, int64_t N,
+                          uint64_t seed, void *dx_bf16, void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
+                          qt2_stream_t stream) {
+    if (!dy || !x || !w || !dx_bf16 || !dw) return QT2_ERR_INVALID_ARG;
+    if (dw_dtype != QT2_DTYPE_BF16 && dw_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    if (!aligned16(dy) || !aligned16(x) || !aligned16(w) || !aligned16(dx_bf16) || !aligned16(dw))
+        return QT2_ERR_ALIGN;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    BwdLayout L;
+    if (ws_bytes < linear_bwd_layout(M, K, N, workspace, &L)) return QT2_ERR_WORKSPACE;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // dY: both views from one read; W and X: column views (rotated along N and M respectively)
+    if ((st = msed_enqueue(dy, M, N, N, QT2_LAYOUT_BOTH, seed, QT2_TID_DY_ROW, QT2_TID_DY_COL, L.dy_row, L.dy_col,
+                           L.P_dy_row, L.P_dy_col, L.amax, s)) != QT2_OK)
+        return st;
+    const DevView none{nullptr, nullptr, nullptr};
+    if ((st = msed_enqueue(w, N, K, K, QT2_LAYOUT_COL, seed, 0, QT2_TID_W_COL, none, L.w_col, nullptr, L.P_w_col,
+                           L.amax + 2, s)) != QT2_OK)
+        return st;
+    if ((st = msed_enqueue(x, M, K, K, QT2_LAYOUT_COL, seed, 0, QT2_TID_X_COL, none, L.x_col, nullptr, L.P_x_col,
+                           L.amax + 4, s)) != QT2_OK)
+        return st;
+    // dgrad: dX[M][K] = 2^-7 * dY_row[M][N] . W_col[K][N]^T
+    if ((st = gemm_enqueue(L.dy_row, L.w_col, M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK) return st;
+    // wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
+    return gemm_enqueue(L.dy_col, L.x_col, N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
+}
+
+}  // extern "C"

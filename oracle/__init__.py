@@ -70,6 +70,7 @@ def lib():
                 "or_msedEN_tensor_scale": (f32, [f32]),
                 "or_msedEN_finalize": (None, [vp, i64, i64, f32, u64, u32, i64, i64, vp]),
                 "or_dequant": (None, [vp, vp, i64, i64, f32, i64, i64, vp]),
+                "or_dequant_row": (None, [vp, vp, i64, i64, f32, i64, vp]),
                 "or_unrotate_rows": (None, [vp, i64, i64, vp, i64, i64, vp]),
                 "or_gemm_f64": (None, [vp, vp, i64, i64, i64, f64, i64, i64, vp]),
                 "or_rotated_amax_rows": (f32, [vp, i64, i64, vp, i64, i64]),
@@ -193,6 +194,16 @@ class View:
         R, C = self.shape
         out = np.empty((R, C), dtype=np.float64)
         _rows(lambda r0, r1: lib().or_dequant(_p(self.codes), _p(self.scales), R, C, float(self.g), r0, r1, _p(out)), R)
+        return out
+
+    def dequant_rows(self, rows) -> np.ndarray:
+        """Dequantized rows (fp64) of the given row indices only."""
+        R, C = self.shape
+        out = np.empty((len(rows), C), dtype=np.float64)
+        for i, r in enumerate(rows):
+            row = np.empty(C, dtype=np.float64)
+            lib().or_dequant_row(_p(self.codes), _p(self.scales), R, C, float(self.g), int(r), _p(row))
+            out[i] = row
         return out
 
 

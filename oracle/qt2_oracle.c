@@ -392,6 +392,18 @@ OR_EXPORT void or_dequant(const uint8_t *codes, const uint8_t *scales, int64_t R
         }
 }
 
+/* One dequantized row r (fp64) into out[0..C). */
+OR_EXPORT void or_dequant_row(const uint8_t *codes, const uint8_t *scales, int64_t R, int64_t C, float g, int64_t r,
+                              double *out)
+{
+    (void)R;
+    for (int64_t c = 0; c < C; c++) {
+        uint8_t byte = codes[r * (C / 2) + c / 2];
+        uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+        out[c] = (double)or_e2m1_value(code) * (double)or_e4m3_value(scales[r * (C / 16) + c / 16]) * (double)g;
+    }
+}
+
 /* Inverse rotation of rotated-domain rows (fp64): x = (1/128) D H y per 128-block. */
 OR_EXPORT void or_unrotate_rows(const double *y, int64_t R, int64_t C, const float sgn[128], int64_t r0,
                                 int64_t r1, double *out)

@@ -1,0 +1,109 @@
+"""The C-ABI library builds for sm_100a, loads, exports every function include/qt2.h declares,
+and rejects bad arguments on the host before any CUDA work (CPU only: no compute call needs a
+GPU here; without one, a valid call must fail with QT2_ERR_DEVICE, never fall back)."""
+import ctypes
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_quantized_b200 import build as qbuild
+from nvfp4_quantized_b200 import qt2
+from tests.layout import canonical_to_scales, scale_offsets, scales_to_canonical
+
+
+@pytest.fixture(scope="module")
+def L():
+    qbuild.build()
+    return qt2.lib()
+
+
+def test_exports_every_header_function(L):
+    names = qt2.header_functions()
+    assert len(names) == 12
+    out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)
+    # nothing but the C ABI leaks out of the library
+    assert {e for e in exported if e.startswith("qt2")} == set(names)
+
+
+def test_built_for_sm100a_only():
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", qt2.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    assert "sm_100a" in out and "sm_90" not in out
+
+
+def test_version_and_status_strings(L):
+    assert qt2.qt2_version() >= 100
+    for code in range(0, -8, -1):
+        s = qt2.qt2_status_string(code)
+        assert s and s != "unknown status"
+
+
+def test_workspace_size_queries(L):
+    M, K, N = 256, 512, 384
+    fwd = qt2.qt2_linear_fwd_workspace_size(M, K, N)
+    view = lambda R, C: (R * C // 2 + 255) // 256 * 256 + (R * C // 16 + 255) // 256 * 256 + 256
+    assert fwd == 256 + view(M, K) + view(N, K)
+    bwd = qt2.qt2_linear_bwd_workspace_size(M, K, N)
+    assert bwd >= view(M, N) * 2 + view(K, N) + view(K, M) + 4 * (M * N + N * K + M * K) // 16
+    assert qt2.qt2_quant_msedEN_workspace_size(M, K, qt2.QT2_LAYOUT_BOTH) == 256 + 2 * (M * K // 16 * 4)
+    with pytest.raises(qt2.QT2Error) as e:
+        qt2.qt2_linear_fwd_workspace_size(100, 128, 128)
+    assert e.value.status == qt2.QT2_ERR_SHAPE
+
+
+def _view(codes=0x10000, scales=0x20000, ts=0x30000):
+    return qt2.NVFP4ViewC(codes, scales, ts)
+
+
+def test_host_validation_codes(L):
+    """Fake, never-dereferenced device addresses: validation happens before any CUDA call."""
+    v = _view()
+    f = L.qt2_quant_fwd46
+    R = ctypes.byref
+    assert f(None, 128, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_INVALID_ARG
+    assert f(0x1000, 100, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
+    assert f(0x1000, 128, 128, 64, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
+    assert f(0x1008, 128, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
+    assert f(0x1000, 128, 128, 132, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
+    assert f(0x1000, 128, 128, 128, 2, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_INVALID_ARG
+    assert f(0x1000, 128, 128, 128, 1, R(v), None, None, 256, None) == qt2.QT2_ERR_WORKSPACE
+    assert f(0x1000, 128, 128, 128, 1, R(_view(codes=0x10008)), None, 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
+    g = L.qt2_quant_msedEN
+    assert g(0x1000, 128, 128, 128, 0, 1, 1, 2, R(v), R(v), 0x40000, 1 << 20, None) == qt2.QT2_ERR_INVALID_ARG
+    assert g(0x1000, 128, 128, 128, 3, 1, 1, 2, R(v), None, 0x40000, 1 << 20, None) == qt2.QT2_ERR_INVALID_ARG
+    assert g(0x1000, 128, 128, 128, 3, 1, 1, 2, R(v), R(v), 0x40000, 16, None) == qt2.QT2_ERR_WORKSPACE
+    assert g(0x1000, 128, 128, 128, 3, 1, 1, 2, R(v), R(v), 0x40010, 1 << 20, None) == qt2.QT2_ERR_ALIGN
+    h = L.qt2_gemm_nvfp4
+    assert h(R(v), R(v), 128, 128, 128, 1.0, None, 0, 128, None) == qt2.QT2_ERR_INVALID_ARG
+    assert h(R(v), R(v), 128, 128, 128, 1.0, 0x50000, 7, 128, None) == qt2.QT2_ERR_INVALID_ARG
+    assert h(R(v), R(v), 128, 192, 128, 1.0, 0x50000, 0, 192, None) == qt2.QT2_ERR_SHAPE
+    assert h(R(v), R(v), 128, 128, 128, 1.0, 0x50000, 0, 64, None) == qt2.QT2_ERR_SHAPE
+    assert L.qt2_linear_fwd(0x1000, 0x2000, 128, 128, 128, 0x3000, None, 0, None) == qt2.QT2_ERR_WORKSPACE
+    assert L.qt2_linear_bwd(0x1000, 0x2000, 0x3000, 128, 128, 128, 0, 0x4000, 0x5000, 3, 0x6000, 1 << 30,
+                            None) == qt2.QT2_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_valid_call_without_gpu_fails_loudly(L):
+    v = _view()
+    st = L.qt2_quant_fwd46(0x1000, 128, 128, 128, 1, ctypes.byref(v), None, 0x40000, 256, None)
+    assert st == qt2.QT2_ERR_DEVICE
+    with pytest.raises(qt2.QT2Error):
+        qt2._check("qt2_quant_fwd46", st)
+
+
+def test_scale_layout_helpers_are_inverse():
+    R, C = 256, 512
+    off = scale_offsets(R, C)
+    assert sorted(off.ravel().tolist()) == list(range(R * C // 16))
+    canon = np.random.default_rng(0).integers(0, 127, (R, C // 16)).astype(np.uint8)
+    assert np.array_equal(scales_to_canonical(canonical_to_scales(canon), R, C), canon)
+    # one 512-byte atom holds 128 rows x 4 groups; rows r, r+32, r+64, r+96 share a 16-byte line
+    assert off[0, 0] == 0 and off[32, 0] == 4 and off[1, 0] == 16 and off[0, 1] == 1 and off[0, 4] == 512

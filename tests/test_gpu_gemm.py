@@ -1,0 +1,82 @@
+"""GPU parity of the block-scaled NVFP4 GEMM: the tcgen05 kernel (through the C ABI) consumes
+views produced by the oracle and is compared with the oracle's fp64 product of the dequantized
+operands.  Bar (fp32 output): relative Frobenius error <= 1e-5 and, elementwise,
+|err| <= 1e-4 * sum_k |a_ik| |b_jk|.  bf16 output adds its own rounding (2^-9 relative)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_quantized_b200 import qt2
+from tests.layout import canonical_to_scales
+
+pytestmark = pytest.mark.gpu
+
+
+def upload(view: O.View) -> qt2.View:
+    return qt2.View(torch.from_numpy(view.codes).cuda(), torch.from_numpy(canonical_to_scales(view.scales)).cuda(),
+                    torch.tensor([float(view.g)], dtype=torch.float32).cuda())
+
+
+def gpu_gemm(va: O.View, vb: O.View, alpha: float, dtype: int):
+    M, K = va.shape
+    N = vb.shape[0]
+    out = torch.empty((M, N), dtype=torch.float32 if dtype == qt2.QT2_DTYPE_F32 else torch.bfloat16, device="cuda")
+    a, b = upload(va), upload(vb)
+    qt2.qt2_gemm_nvfp4(a, b, M, N, K, alpha, out, dtype, N)
+    assert qt2.qt2_device_status() == 0
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+def check(got, va, vb, alpha, bf16=False):
+    A, B = va.dequant(), vb.dequant()
+    ref = O.gemm(A, B, alpha)
+    bound = O.gemm(np.abs(A), np.abs(B), abs(alpha))
+    err = np.abs(got - ref)
+    if bf16:
+        assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-4 * bound + 1e-30)
+        assert np.linalg.norm(got - ref) <= 4e-3 * np.linalg.norm(ref) + 1e-30
+    else:
+        assert np.all(err <= 1e-4 * bound + 1e-30), np.max(err / (bound + 1e-30))
+        assert np.linalg.norm(got - ref) <= 1e-5 * np.linalg.norm(ref) + 1e-30, \
+            np.linalg.norm(got - ref) / np.linalg.norm(ref)
+
+
+def _x(R, C, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((R, C), generator=g) * scale).to(torch.bfloat16)
+
+
+# (M, N, K): single tile, N % 256 != 0 (128-wide tiles), K not a multiple of 256 (half stage),
+# several stages around the ring, a long K.
+SHAPES = [(128, 128, 128), (128, 256, 256), (256, 256, 256), (384, 640, 1152), (256, 512, 2048), (128, 384, 4224),
+          (256, 256, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("dtype", [qt2.QT2_DTYPE_F32, qt2.QT2_DTYPE_BF16])
+def test_gemm_forward_operands(M, N, K, dtype):
+    va = O.fwd46(_x(M, K, 1))
+    vb = O.fwd46(_x(N, K, 2, 0.02))
+    got = gpu_gemm(va, vb, 1.0, dtype)
+    check(got, va, vb, 1.0, bf16=dtype == qt2.QT2_DTYPE_BF16)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (384, 640, 1152), (128, 384, 4224)])
+def test_gemm_msedEN_operands(M, N, K):
+    seed = 5
+    va = O.msedEN(_x(M, K, 3, 1e-4), seed, 1, "row")
+    vb = O.msedEN(_x(N, K, 4, 0.02), seed, 3, "row")
+    got = gpu_gemm(va, vb, 2.0 ** -7, qt2.QT2_DTYPE_F32)
+    check(got, va, vb, 2.0 ** -7)
+
+
+def test_gemm_zero_and_extreme_scales():
+    M = N = K = 256
+    x = _x(M, K, 6)
+    x[:128] = 0.0
+    va = O.fwd46(x)
+    vb = O.fwd46(_x(N, K, 7) * 3e4)
+    got = gpu_gemm(va, vb, 1.0, qt2.QT2_DTYPE_F32)
+    assert np.all(got[:128] == 0.0)
+    check(got, va, vb, 1.0)

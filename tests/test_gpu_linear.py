@@ -1,0 +1,126 @@
+"""GPU parity of the composed linear layer (qt2_linear_fwd / qt2_linear_bwd through the C ABI)
+against the oracle's fp64 results on the same seeded inputs.
+
+Small cases compare every output; the full-size case (the 1.9B-class layer: tokens 16384,
+d_in 2048, d_out 8192, the launch configuration the benchmark times) compares sampled rows
+that the oracle computes one by one, plus bit-exact codes and scales of those rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from nvfp4_quantized_b200 import qt2
+from nvfp4_quantized_b200 import synth
+from tests.layout import scales_to_canonical
+
+pytestmark = pytest.mark.gpu
+
+
+def run_linear(x, w, dy, seed, dw_dtype=qt2.QT2_DTYPE_F32):
+    M, K = x.shape
+    N = w.shape[0]
+    xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32 if dw_dtype == qt2.QT2_DTYPE_F32 else torch.bfloat16, device="cuda")
+    wsf = qt2.alloc_workspace(qt2.qt2_linear_fwd_workspace_size(M, K, N))
+    wsb = qt2.alloc_workspace(qt2.qt2_linear_bwd_workspace_size(M, K, N))
+    qt2.qt2_linear_fwd(xd, wd, M, K, N, y, wsf, wsf.numel())
+    qt2.qt2_linear_bwd(dyd, xd, wd, M, K, N, seed, dx, dw, dw_dtype, wsb, wsb.numel())
+    assert qt2.qt2_device_status() == 0
+    return y, dx, dw
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+def _bound_check(got, ref, bound, bf16):
+    err = np.abs(got - ref)
+    tol = 1e-4 * bound + (2.0 ** -8 * np.abs(ref) if bf16 else 0.0) + 1e-30
+    assert np.all(err <= tol), np.max(err / tol)
+
+
+@pytest.mark.parametrize("shape,seed", [((256, 256, 256), 0), ((384, 640, 1152), 1), ((512, 384, 256), 2)])
+def test_linear_matches_oracle(shape, seed):
+    M, K, N = shape
+    if shape == (256, 256, 256):
+        x, w, dy = synth.linear_inputs("tiny", seed)
+    else:
+        x, w, dy = synth.custom_linear_inputs(M, K, N, seed)
+    y, dx, dw = run_linear(x, w, dy, seed=1234 + seed)
+    y_ref, vx, vw = O.linear_fwd(x, w)
+    dx_ref, dw_ref, views = O.linear_bwd(dy, x, w, 1234 + seed)
+
+    y_g = y.float().cpu().numpy().astype(np.float64)
+    assert _rel(y_g, y_ref) < 4e-3
+    _bound_check(y_g, y_ref, O.gemm(np.abs(vx.dequant()), np.abs(vw.dequant())), True)
+
+    dx_g = dx.float().cpu().numpy().astype(np.float64)
+    assert _rel(dx_g, dx_ref) < 4e-3
+    _bound_check(dx_g, dx_ref, O.gemm(np.abs(views["dy_row"].dequant()), np.abs(views["w_col"].dequant()), 2 ** -7),
+                 True)
+
+    dw_g = dw.cpu().numpy().astype(np.float64)
+    assert _rel(dw_g, dw_ref) < 1e-5
+    _bound_check(dw_g, dw_ref, O.gemm(np.abs(views["dy_col"].dequant()), np.abs(views["x_col"].dequant()), 2 ** -7),
+                 False)
+
+
+def test_linear_bwd_bf16_dw():
+    x, w, dy = synth.linear_inputs("tiny", 3)
+    _, _, dw = run_linear(x, w, dy, seed=9, dw_dtype=qt2.QT2_DTYPE_BF16)
+    _, dw_ref, _ = O.linear_bwd(dy, x, w, 9)
+    assert _rel(dw.float().cpu().numpy().astype(np.float64), dw_ref) < 4e-3
+
+
+def _view_rows(view: qt2.View, rows, R, C):
+    codes = view.codes[torch.from_numpy(rows).cuda()].cpu().numpy()
+    scales = scales_to_canonical(view.scales.cpu().numpy(), R, C)[rows]
+    return codes, scales, np.float32(view.tensor_scale.item())
+
+
+def test_full_size_llm1p9b_sampled():
+    """Tokens 16384, d_in 2048, d_out 8192: sampled rows of Y, dX and dW against the oracle, and
+    bit-exact codes/scales of the sampled rows of every quantized view."""
+    M, K, N = synth.SHAPES["llm1p9b"]
+    x, w, dy = synth.linear_inputs("llm1p9b", 0)
+    seed = 2024
+    y, dx, dw = run_linear(x, w, dy, seed)
+    rng = np.random.default_rng(0)
+    rows_m = np.sort(rng.choice(M, 6, replace=False))
+    rows_n = np.sort(rng.choice(N, 6, replace=False))
+
+    # forward: X rows via the oracle's row-range quantizer with the full-tensor max; W in full
+    vx_full = O.fwd46(x)       # all rows (cheap enough: 33M elements)
+    vw = O.fwd46(w)
+    y_ref = O.gemm(vx_full.dequant_rows(rows_m), vw.dequant(), 1.0)
+    y_g = y[torch.from_numpy(rows_m).cuda()].float().cpu().numpy().astype(np.float64)
+    assert _rel(y_g, y_ref) < 4e-3
+
+    # standalone quantizers at full size, same launch configuration as inside the layer
+    xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
+    v_dy_row, v_dy_col = qt2.alloc_view(M, N), qt2.alloc_view(N, M)
+    ws = qt2.alloc_workspace(qt2.qt2_quant_msedEN_workspace_size(M, N, qt2.QT2_LAYOUT_BOTH))
+    qt2.qt2_quant_msedEN(dyd, M, N, N, qt2.QT2_LAYOUT_BOTH, seed, qt2.QT2_TID_DY_ROW, qt2.QT2_TID_DY_COL, v_dy_row,
+                         v_dy_col, ws, ws.numel())
+    assert qt2.qt2_device_status() == 0
+
+    o_dy_row = O.msedEN(dy, seed, qt2.QT2_TID_DY_ROW, "row")
+    o_w_col = O.msedEN(w, seed, qt2.QT2_TID_W_COL, "col")
+    got = _view_rows(v_dy_row, rows_m, M, N)
+    assert got[2] == o_dy_row.g
+    assert np.array_equal(got[0], o_dy_row.codes[rows_m]) and np.array_equal(got[1], o_dy_row.scales[rows_m])
+    dx_ref = O.gemm(o_dy_row.dequant_rows(rows_m), o_w_col.dequant(), 2.0 ** -7)
+    dx_g = dx[torch.from_numpy(rows_m).cuda()].float().cpu().numpy().astype(np.float64)
+    assert _rel(dx_g, dx_ref) < 4e-3
+    del o_dy_row
+
+    o_dy_col = O.msedEN(dy, seed, qt2.QT2_TID_DY_COL, "col")
+    o_x_col = O.msedEN(x, seed, qt2.QT2_TID_X_COL, "col")
+    got = _view_rows(v_dy_col, rows_n, N, M)
+    assert got[2] == o_dy_col.g
+    assert np.array_equal(got[0], o_dy_col.codes[rows_n]) and np.array_equal(got[1], o_dy_col.scales[rows_n])
+    dw_ref = O.gemm(o_dy_col.dequant_rows(rows_n), o_x_col.dequant(), 2.0 ** -7)
+    dw_g = dw[torch.from_numpy(rows_n).cuda()].cpu().numpy().astype(np.float64)
+    assert _rel(dw_g, dw_ref) < 1e-5
