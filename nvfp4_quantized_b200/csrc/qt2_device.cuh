@@ -52,23 +52,21 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     return r;
 }
 
+// Two E2M1 codes in the low byte of `byte` -> f16x2 (low nibble -> low half).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "r"(byte));
+    return h2;
+}
+
 // Eight packed E2M1 codes -> their exact values as fp32 (nibble i -> out[i]).
 __device__ __forceinline__ void e2m1x8_values(uint32_t codes, float (&out)[8]) {
-    uint32_t h0, h1, h2, h3;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-        : "r"(codes));
-    const uint32_t h[4] = {h0, h1, h2, h3};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+        const uint32_t h = e2m1x2_to_f16x2(codes >> (8 * i));
         asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
             : "=f"(out[2 * i]), "=f"(out[2 * i + 1])
-            : "r"(h[i]));
+            : "r"(h));
     }
 }
 
