@@ -1,0 +1,396 @@
+"""Benchmark of the Quartet II NVFP4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config llm1p9b]
+
+A step is one pass of the whole hot path over one batch: the forward quantizer on X and W
+(tensor max + RTN/4-6), the forward GEMM, MS-EDEN on dY (row and column views in one pass),
+on W (column view) and on X (column view) with their scale passes, and the dgrad and wgrad
+GEMMs -- the calls qt2_linear_fwd + qt2_linear_bwd make, issued here one C-ABI call at a time
+so that each kernel's duration is taken with CUDA events inside the timed region.
+
+Workload (default): the 1.9B-class layer, tokens 16384 x d_in 2048 -> d_out 8192, bf16 inputs
+drawn by nvfp4_quantized_b200.synth (seeded, synthetic).  Two input sets alternate between
+steps (704 MiB > L2), so no step starts with its inputs in L2.
+
+Multi-GPU (torchrun, one rank per GPU): the path has no exchange step, so every rank runs the
+same step on its own token batch (weak scaling, no collective on the data path); the time is
+the max over ranks and value = all ranks' FLOPs / that time.
+
+--impl reference times the CPU oracle (the plain restatement the CUDA path is checked
+against) on a bounded sample of the same workload, on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Quartet II linear fwd+bwd TFLOPS; quantizer GB/s; % of FP4/HBM roofline"
+UNIT = "TFLOP/s"
+KERNELS_PER_STEP = 14   # amax x2, fwd46 x2, gemm x3, MS-EDEN tiles x3, scale finalize x4
+
+# Algorithmic bytes per input element of each quantizer call (reads + writes the method needs).
+BYTES_FWD46 = 2 + 2 + 0.5 + 1 / 16            # max pass read, quantize read, codes, scales
+BYTES_MSED_ONE = 2 + 0.5 + 0.25 + 0.25 + 1 / 16  # read, codes, pre-scale write + read, scales
+BYTES_MSED_BOTH = 2 + 2 * (0.5 + 0.25 + 0.25 + 1 / 16)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples the SM clock, power and clock-event reasons through NVML every few ms while the
+    timed region runs (read-only queries; no setting is touched)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index: int, period_s: float = 0.005):
+        self.gpu, self.period = gpu_index, period_s
+        self.samples = []
+        self._stop = None
+
+    def _run(self):
+        import pynvml
+        try:
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, pw, rs))
+                self._stop.wait(self.period)
+        except Exception as e:   # NVML unavailable: report that, never fail the run
+            self.error = repr(e)
+
+    def __enter__(self):
+        import threading
+        self.max_mhz, self.error = None, None
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0,
+                    "error": self.error}
+        loaded = [s for s in self.samples if s[1] > 250.0] or self.samples
+        sm = sorted(s[0] for s in loaded)
+        reasons = sorted({n for s in loaded for n, bit in self.REASONS.items() if s[2] & bit})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "samples_under_load": len(loaded),
+                "power_w_max": max(s[1] for s in self.samples), "source": "nvml, 5 ms period"}
+
+
+# ---------------------------------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from nvfp4_quantized_b200 import qt2, synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M, K, N = synth.SHAPES[args.config]
+    Q = qt2
+    ROW, COL, BOTH = Q.QT2_LAYOUT_ROW, Q.QT2_LAYOUT_COL, Q.QT2_LAYOUT_BOTH
+
+    # two resident input sets (seeded per rank), outputs and every intermediate view
+    sets = []
+    for i in range(2):
+        x, w, dy = synth.linear_inputs(args.config, seed=1000 * rank + 10 * i, device=dev)
+        sets.append((x, w, dy))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((N, K), dtype=torch.float32, device=dev)
+    vx, vw = Q.alloc_view(M, K, dev), Q.alloc_view(N, K, dev)
+    v_dy_row, v_dy_col = Q.alloc_view(M, N, dev), Q.alloc_view(N, M, dev)
+    v_w_col, v_x_col = Q.alloc_view(K, N, dev), Q.alloc_view(K, M, dev)
+    ws46 = Q.alloc_workspace(Q.qt2_quant_fwd46_workspace_size(max(M, N), K), dev)
+    ws46b = Q.alloc_workspace(Q.qt2_quant_fwd46_workspace_size(max(M, N), K), dev)
+    ws_dy = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(M, N, BOTH), dev)
+    ws_w = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(N, K, COL), dev)
+    ws_x = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(M, K, COL), dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["fwd46_x", "fwd46_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col", "gemm_dgrad",
+             "gemm_wgrad"]
+
+    def step(i, ev=None):
+        x, w, dy = sets[i % 2]
+        seed = 0x5EED0000 + i
+
+        def mark(j):
+            if ev is not None:
+                ev[j].record(stream)
+        mark(0)
+        Q.qt2_quant_fwd46(x, M, K, K, ROW, vx, None, ws46, ws46.numel(), stream)
+        mark(1)
+        Q.qt2_quant_fwd46(w, N, K, K, ROW, vw, None, ws46b, ws46b.numel(), stream)
+        mark(2)
+        Q.qt2_gemm_nvfp4(vx, vw, M, N, K, 1.0, y, Q.QT2_DTYPE_BF16, N, stream)
+        mark(3)
+        Q.qt2_quant_msedEN(dy, M, N, N, BOTH, seed, Q.QT2_TID_DY_ROW, Q.QT2_TID_DY_COL, v_dy_row, v_dy_col, ws_dy,
+                           ws_dy.numel(), stream)
+        mark(4)
+        Q.qt2_quant_msedEN(w, N, K, K, COL, seed, 0, Q.QT2_TID_W_COL, None, v_w_col, ws_w, ws_w.numel(), stream)
+        mark(5)
+        Q.qt2_quant_msedEN(x, M, K, K, COL, seed, 0, Q.QT2_TID_X_COL, None, v_x_col, ws_x, ws_x.numel(), stream)
+        mark(6)
+        Q.qt2_gemm_nvfp4(v_dy_row, v_w_col, M, K, N, 2.0 ** -7, dx, Q.QT2_DTYPE_BF16, K, stream)
+        mark(7)
+        Q.qt2_gemm_nvfp4(v_dy_col, v_x_col, N, K, M, 2.0 ** -7, dw, Q.QT2_DTYPE_F32, K, stream)
+        mark(8)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert Q.qt2_device_status(stream) == 0, "device status word set during warm-up"
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    status = Q.qt2_device_status(stream)
+    per = {n: sum(events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)) / args.steps
+           for j, n in enumerate(names)}
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # ------------------------------------------------------------------ end to end through the API
+    e2e = None
+    if not args.no_e2e:
+        hx = sets[0][0].cpu().pin_memory()
+        hw = sets[0][1].cpu().pin_memory()
+        hdy = sets[0][2].cpu().pin_memory()
+        hy = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        hdx = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+        hdw = torch.empty((N, K), dtype=torch.float32).pin_memory()
+        dxi, dwi, ddyi = torch.empty_like(sets[0][0]), torch.empty_like(sets[0][1]), torch.empty_like(sets[0][2])
+        wsf = Q.alloc_workspace(Q.qt2_linear_fwd_workspace_size(M, K, N), dev)
+        wsb = Q.alloc_workspace(Q.qt2_linear_bwd_workspace_size(M, K, N), dev)
+
+        def e2e_step(i):
+            dxi.copy_(hx, non_blocking=True)
+            dwi.copy_(hw, non_blocking=True)
+            ddyi.copy_(hdy, non_blocking=True)
+            Q.qt2_linear_fwd(dxi, dwi, M, K, N, y, wsf, wsf.numel(), stream)
+            Q.qt2_linear_bwd(ddyi, dxi, dwi, M, K, N, 0xE2E0 + i, dx, dw, Q.QT2_DTYPE_F32, wsb, wsb.numel(), stream)
+            hy.copy_(y, non_blocking=True)
+            hdx.copy_(dx, non_blocking=True)
+            hdw.copy_(dw, non_blocking=True)
+
+        for i in range(min(args.warmup, 3)):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier()
+        e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_s.record(stream)
+        n_e2e = max(1, min(args.steps, 10))
+        for i in range(n_e2e):
+            e2e_step(100 + i)
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        flops_step = 3 * 2.0 * M * N * K
+        e2e = {"value": world * flops_step * n_e2e / (float(te.item()) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": hx.numel() * 2 + hw.numel() * 2 + hdy.numel() * 2,
+               "d2h_bytes_per_step": hy.numel() * 2 + hdx.numel() * 2 + hdw.numel() * 4,
+               "steps": n_e2e, "ms_per_step": float(te.item()) / n_e2e}
+    return dict(M=M, K=K, N=N, max_ms=max_ms, per=per, status=status, clocks=clk.summary(), e2e=e2e)
+
+
+def cpu_baseline(config: str, tokens: int = 256):
+    """The oracle, as it stands, on a bounded sample of the workload: the full step restricted
+    to `tokens` rows of X and dY (W in full).  Returns (TFLOP/s, seconds, cores, sample)."""
+    import oracle as O
+    from nvfp4_quantized_b200 import synth
+
+    M, K, N = synth.SHAPES[config]
+    x, w, dy = synth.linear_inputs(config, seed=0)
+    xs, dys = x[:tokens].contiguous(), dy[:tokens].contiguous()
+    O.build()
+    t0 = time.perf_counter()
+    O.linear_fwd(xs, w)
+    O.linear_bwd(dys, xs, w, seed=1)
+    dt = time.perf_counter() - t0
+    flops = 3 * 2.0 * tokens * N * K
+    sample = (f"full fwd+bwd step on {tokens} of {M} tokens (X, dY rows), W {N}x{K} in full; "
+              f"oracle fp64 GEMMs and bit-exact quantizers")
+    return flops / dt / 1e12, dt, O.threads(), sample
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="llm1p9b")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--cpu-tokens", type=int, default=2048)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from nvfp4_quantized_b200 import synth
+    M, K, N = synth.SHAPES[args.config]
+    workload = (f"Quartet II NVFP4 linear layer fwd+bwd (forward RTN+4/6, backward MS-EDEN, 3 block-scaled "
+                f"GEMMs): tokens {M}, d_in {K}, d_out {N}")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = []
+        for i in range(args.warmup + args.steps):
+            v, dt, cores, sample = cpu_baseline(args.config, args.ref_tokens)
+            if i >= args.warmup:
+                steps.append((v, dt))
+        value = sum(v for v, _ in steps) / len(steps)
+        ms = 1e3 * sum(dt for _, dt in steps) / len(steps)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (GEMM), f32 (quantizers)",
+                "data": "synthetic", "config": {"workload": workload, "sample_tokens": args.ref_tokens},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    from nvfp4_quantized_b200 import build as qbuild
+    if rank == 0:
+        qbuild.build()
+    if world > 1:
+        dist.barrier()
+
+    r = run_ours(args, rank, world, local_rank)
+    pk = peaks()
+    flops_gemm = 2.0 * M * N * K
+    flops_step = 3 * flops_gemm
+    value = world * flops_step * args.steps / (r["max_ms"] * 1e-3) / 1e12
+    per = r["per"]
+    gemm_ms = (per["gemm_fwd"] + per["gemm_dgrad"] + per["gemm_wgrad"]) / 3
+    fp4_peak = pk["bf16_sustained"] * 4.0
+    achieved = flops_gemm / (gemm_ms * 1e-3) / 1e12
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "gemm_nvfp4_traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                tj = json.load(f)
+            import hashlib
+            src = os.path.join(ROOT, "nvfp4_quantized_b200", "csrc", "gemm_kernel.cuh")
+            sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+            if tj.get("config") == args.config and tj.get("kernel_sha1") == sha:
+                traffic = tj.get("bytes_per_launch")   # counters of the current kernel only
+        except Exception:
+            traffic = None
+
+    def gbs(bytes_, ms):
+        return bytes_ / (ms * 1e-3) / 1e9
+
+    kernels = {
+        "gemm_fwd": {"ms": per["gemm_fwd"], "tflops": flops_gemm / (per["gemm_fwd"] * 1e-3) / 1e12},
+        "gemm_dgrad": {"ms": per["gemm_dgrad"], "tflops": flops_gemm / (per["gemm_dgrad"] * 1e-3) / 1e12},
+        "gemm_wgrad": {"ms": per["gemm_wgrad"], "tflops": flops_gemm / (per["gemm_wgrad"] * 1e-3) / 1e12},
+        "fwd46_x": {"ms": per["fwd46_x"], "gbs": gbs(M * K * BYTES_FWD46, per["fwd46_x"])},
+        "fwd46_w": {"ms": per["fwd46_w"], "gbs": gbs(N * K * BYTES_FWD46, per["fwd46_w"])},
+        "msed_dy_both": {"ms": per["msed_dy_both"], "gbs": gbs(M * N * BYTES_MSED_BOTH, per["msed_dy_both"])},
+        "msed_w_col": {"ms": per["msed_w_col"], "gbs": gbs(N * K * BYTES_MSED_ONE, per["msed_w_col"])},
+        "msed_x_col": {"ms": per["msed_x_col"], "gbs": gbs(M * K * BYTES_MSED_ONE, per["msed_x_col"])},
+    }
+    for k, v in kernels.items():
+        if "gbs" in v:
+            v["hbm_frac"] = v["gbs"] / pk["hbm_gbs"]
+        else:
+            v["fp4_frac"] = v["tflops"] / fp4_peak
+    quant_ms = sum(per[n] for n in names_quant())
+    quant_bytes = (M * K + N * K) * BYTES_FWD46 + M * N * BYTES_MSED_BOTH + (N * K + M * K) * BYTES_MSED_ONE
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": r["max_ms"] / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x ue4m3 block-scaled GEMM, fp32 accumulate; fp32 quantizers)",
+        "data": "synthetic (seeded bf16 tensors with the layer's distributions)",
+        "config": {"workload": workload, "M": M, "K": K, "N": N,
+                   "parallelism": f"dp{world}: every rank its own token batch, no collective on the path",
+                   "l2": "inputs larger than L2: two 352 MiB input sets alternate between steps",
+                   "output": "Y bf16, dX bf16, dW fp32"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp4_peak, "traffic": traffic,
+                     "kernel": "gemm_nvfp4 (mean of the fwd, dgrad and wgrad launches)",
+                     "peak_source": f"{pk['source']}: sustained bf16 {pk['bf16_sustained']} TFLOP/s x 4 "
+                                    "(nominal dense fp4/bf16 ratio)"},
+        "quantizers": {"gbs": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                       "hbm_frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                       "peak_gbs": pk["hbm_gbs"], "ms_per_step": quant_ms},
+        "kernels": kernels,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    if r["e2e"] is not None:
+        line["e2e"] = r["e2e"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, cores, sample = cpu_baseline(args.config, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def names_quant():
+    return ["fwd46_x", "fwd46_w", "msed_dy_both", "msed_w_col", "msed_x_col"]
+
+
+if __name__ == "__main__":
+    main()
