@@ -129,6 +129,31 @@ QT2_API qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t co
                             size_t ws_bytes, qt2_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * MS-EDEN without a workspace.  The Quartet II pages have no counterpart to this call; it is a
+ * convenience of this library for callers that cannot allocate device memory for scratch (a
+ * runtime that has handed all device memory to its own pools, a latency-critical path that
+ * must not call cudaMalloc, a plugin whose host framework owns the allocator).
+ *
+ * Same arguments and results as qt2_quant_msedEN (bit-identical outputs), minus the
+ * workspace: the scratch lives in a fixed device array of QT2_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * inside the library, which every GPU that loads the library holds until the process exits.
+ * A call needs 256 bytes plus rows*cols/4 bytes per requested view, so at most about 64 Mi
+ * elements with QT2_LAYOUT_BOTH or 128 Mi elements with one view (for example 8192 x 8192
+ * both views); larger tensors return QT2_ERR_WORKSPACE and enqueue nothing.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.
+ * All calls on a device share the one array: the call zeroes the view maxima it needs and
+ * rewrites every pre-scale before reading it, but two calls whose work overlaps on the GPU
+ * (different streams without ordering between them) race on the array and give wrong results.
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine is called.
+ * --------------------------------------------------------------------------------------- */
+#define QT2_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+QT2_API qt2_status qt2_quant_msedEN_noalloc(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                            int layout_mask, uint64_t seed, uint32_t tensor_id_row,
+                                            uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
+                                            const qt2_nvfp4_view *col_out, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * Block-scaled NVFP4 GEMM on the 5th-generation tensor cores ([QII-th] abstract and §1: NVFP4 is
  * natively supported by Blackwell GPUs).  "TN": a is an [M][K] view, b an [N][K] view, both
  * grouped along K.  c[m][n] = alpha * gA * gB * sum_k val(a)*sa * val(b)*sb, accumulated in fp32,

@@ -29,7 +29,7 @@ def sources():
 def nvcc_cmd(out: str, verbose: bool = False):
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "--fmad=false", "-std=c++17",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-o", out, os.path.join(CSRC, "qt2_lib.cu")]
+           "-o", out, os.path.join(CSRC, "qt2_lib.cu"), os.path.join(CSRC, "qt2_noalloc.cu")]
     if verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     return cmd

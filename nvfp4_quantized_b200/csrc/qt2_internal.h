@@ -41,4 +41,14 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, De
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
 
+// Hooks used by the workspace-free MS-EDEN entry point (qt2_noalloc.cu).
+qt2_status msed_check_args(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                           const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out);
+size_t msed_scratch_bytes(int64_t rows, int64_t cols, int layout_mask);
+qt2_status msed_device_check();
+qt2_status msed_enqueue_on_scratch(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                                   uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
+                                   const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *scratch,
+                                   cudaStream_t stream);
+
 }  // namespace qt2

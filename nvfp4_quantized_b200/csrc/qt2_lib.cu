@@ -310,6 +310,43 @@ size_t linear_bwd_layout(int64_t M, int64_t K, int64_t N, void *ws, BwdLayout *L
 
 }  // namespace
 
+namespace qt2 {
+
+// Hooks for the library's other translation unit (the workspace-free MS-EDEN entry point).
+// They reuse the checks and the enqueue sequence of qt2_quant_msedEN on caller-given scratch.
+qt2_status msed_check_args(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                           const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_ROW) && !view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_COL) && !view_ok(col_out)) return col_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    return QT2_OK;
+}
+
+size_t msed_scratch_bytes(int64_t rows, int64_t cols, int layout_mask) {
+    float *a, *b;
+    uint32_t *c;
+    return msed_ws(rows, cols, layout_mask, &a, &b, &c, nullptr);
+}
+
+qt2_status msed_device_check() { return check_device(); }
+
+qt2_status msed_enqueue_on_scratch(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                                   uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
+                                   const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *scratch,
+                                   cudaStream_t stream) {
+    float *P_row, *P_col;
+    uint32_t *amax;
+    msed_ws(rows, cols, layout_mask, &P_row, &P_col, &amax, scratch);
+    const DevView none{nullptr, nullptr, nullptr};
+    return msed_enqueue(x_bf16, rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
+                        (layout_mask & QT2_LAYOUT_ROW) ? dev_view(row_out) : none,
+                        (layout_mask & QT2_LAYOUT_COL) ? dev_view(col_out) : none, P_row, P_col, amax, stream);
+}
+
+}  // namespace qt2
+
 extern "C" {
 
 int qt2_version(void) { return 100; }

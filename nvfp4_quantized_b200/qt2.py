@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
                 "qt2_quant_fwd46": (i32, [vp, i64, i64, i64, i32, pv, pv, vp, sz, vp]),
                 "qt2_quant_msedEN_workspace_size": (i32, [i64, i64, i32, psz]),
                 "qt2_quant_msedEN": (i32, [vp, i64, i64, i64, i32, u64, u32, u32, pv, pv, vp, sz, vp]),
+                "qt2_quant_msedEN_noalloc": (i32, [vp, i64, i64, i64, i32, u64, u32, u32, pv, pv, vp]),
                 "qt2_gemm_nvfp4": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_linear_fwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_fwd": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
@@ -186,6 +187,18 @@ def qt2_quant_msedEN(x: torch.Tensor, rows: int, cols: int, ld: int, layout_mask
     _check("qt2_quant_msedEN", lib().qt2_quant_msedEN(
         _ptr(x), rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
         ctypes.byref(r) if r else None, ctypes.byref(c) if c else None, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def qt2_quant_msedEN_noalloc(x: torch.Tensor, rows: int, cols: int, ld: int, layout_mask: int, seed: int,
+                             tensor_id_row: int, tensor_id_col: int, row_out: View | None, col_out: View | None,
+                             stream=None) -> None:
+    """qt2_quant_msedEN without a workspace: the library's built-in scratch array is used
+    (see include/qt2.h for its size limit and the rule that calls must not overlap)."""
+    r = row_out.c() if row_out is not None else None
+    c = col_out.c() if col_out is not None else None
+    _check("qt2_quant_msedEN_noalloc", lib().qt2_quant_msedEN_noalloc(
+        _ptr(x), rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
+        ctypes.byref(r) if r else None, ctypes.byref(c) if c else None, _stream(stream)))
 
 
 def qt2_gemm_nvfp4(a: View, b: View, M: int, N: int, K: int, alpha: float, c: torch.Tensor, c_dtype: int,
