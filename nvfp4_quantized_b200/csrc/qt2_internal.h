@@ -37,6 +37,11 @@ cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uin
 cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
                               int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s);
 
+cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
+                                   const CUtensorMap &tmSFB, const CUtensorMap &tmC, DevView a, DevView b, int64_t M,
+                                   int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
+                                   cudaStream_t s);
+
 // 2D tensor map for TMA (no multicast anywhere in this library).
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);

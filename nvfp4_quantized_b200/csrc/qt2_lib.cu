@@ -14,7 +14,9 @@
 #include "qt2_internal.h"
 #include "qt2_device.cuh"
 #include "quant_kernels.cuh"
+#include "msed_kernel.cuh"
 #include "gemm_kernel.cuh"
+#include "gemm2_kernel.cuh"
 
 namespace qt2 {
 
@@ -51,22 +53,22 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaGetLastError();
 }
 
-static constexpr int kMsedSmem = 32768 + 1024;
-
-template <bool ROW, bool COL>
+template <int TR, int TC, bool ROW, bool COL>
 static cudaError_t launch_msed_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed, DevView row,
                                        DevView col, float *P_row, float *P_col, uint32_t *amax_row,
                                        uint32_t *amax_col, cudaStream_t s) {
+    constexpr int kSmem = 2 * TR * TC * 2 + 1024;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(msed_tile_kernel<ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kMsedSmem);
+        attr_err = cudaFuncSetAttribute(msed_kernel<TR, TC, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmem);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    dim3 grid((unsigned)(C / 128), (unsigned)(R / 128));
-    msed_tile_kernel<ROW, COL><<<grid, 128, kMsedSmem, s>>>(tmap, R, C, seed, row.codes, P_row, amax_row, col.codes,
-                                                             P_col, amax_col);
+    const int64_t ntiles = (R / TR) * (C / TC);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ntiles, sm_count()));
+    msed_kernel<TR, TC, ROW, COL><<<(unsigned)grid, 256, kSmem, s>>>(tmap, R, C, seed, row.codes, P_row, amax_row,
+                                                                    col.codes, P_col, amax_col);
     return cudaGetLastError();
 }
 
@@ -74,10 +76,20 @@ cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, boo
                               uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
                               uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s) {
     if (do_row && do_col)
-        return launch_msed_variant<true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
-    if (do_row)
-        return launch_msed_variant<true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
-    return launch_msed_variant<false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+        return launch_msed_variant<128, 128, true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
+                                                         s);
+    if (do_row) {
+        if (R % 256 == 0)
+            return launch_msed_variant<256, 128, true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row,
+                                                              amax_col, s);
+        return launch_msed_variant<128, 128, true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row,
+                                                          amax_col, s);
+    }
+    if (C % 256 == 0)
+        return launch_msed_variant<128, 256, false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
+                                                          s);
+    return launch_msed_variant<128, 128, false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
+                                                      s);
 }
 
 cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
@@ -111,6 +123,24 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, De
                               int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s) {
     if (N % 256 == 0) return launch_gemm_bn<256>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
     return launch_gemm_bn<128>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
+}
+
+cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
+                                   const CUtensorMap &tmSFB, const CUtensorMap &tmC, DevView a, DevView b, int64_t M,
+                                   int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
+                                   cudaStream_t s) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        Gemm2Cfg::kSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const int64_t tiles = (M / 256) * (N / 256);
+    const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count() / 2));
+    gemm_nvfp4_pair_kernel<<<(unsigned)(2 * clusters), Gemm2Cfg::kThreads, Gemm2Cfg::kSmemBytes, s>>>(
+        tmA, tmB, tmSFA, tmSFB, tmC, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -262,6 +292,28 @@ qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, 
 qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, float alpha, void *c, int c_dtype,
                         int64_t ldc, cudaStream_t s) {
     CUtensorMap tmA, tmB;
+    if (M % 256 == 0 && N % 256 == 0) {
+        // pair kernel: 128-row code boxes per SM, scale atoms as rows of K/64 512-byte atoms
+        CUtensorMap tmSFA, tmSFB, tmC;
+        if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                            128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b.codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                            128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_tmap_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT64, a.scales, (uint64_t)K, (uint64_t)M / 128,
+                            (uint64_t)K * 8, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT64, b.scales, (uint64_t)K, (uint64_t)N / 128,
+                            (uint64_t)K * 8, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return QT2_ERR_CUDA;
+        // bf16 output leaves through TMA stores of 32-row x 64-column boxes (unused for fp32 output)
+        if (c_dtype == QT2_DTYPE_BF16) {
+            if (!encode_tmap_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c, (uint64_t)N, (uint64_t)M, (uint64_t)ldc * 2,
+                                64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+                return QT2_ERR_CUDA;
+        } else {
+            std::memset(&tmC, 0, sizeof(tmC));
+        }
+        return from_cuda(launch_gemm_nvfp4_pair(tmA, tmB, tmSFA, tmSFB, tmC, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
+    }
     const int bn = (N % 256 == 0) ? 256 : 128;
     if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
                         kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||

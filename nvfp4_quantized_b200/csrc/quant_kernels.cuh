@@ -68,42 +68,83 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint16_t *__restri
 }
 
 // ---------------------------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100a add/sub/mul .f32x2: two IEEE binary32 operations rounded to
+// nearest-even side by side).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// ---------------------------------------------------------------------------------------------
 // Forward quantizer, row view: RTN onto E2M1 with the 4/6 grid choice per 1x16 group
 // ([QII-tg] "Method"; [QII-th] "fairness" answer: the forward pass uses RTN).
 // One thread per 16-element group; a warp covers 32 consecutive groups of one row.
+// Candidate k (6 or 4): s = RNE_E4M3(a/(g*k)), d = s*g, codes = RNE_E2M1(x*(1/d)),
+// err = tree sum of (x - val*d)^2; a zero scale gives sign-preserving zero codes (x*0) and
+// err = sum x^2.  Keep 4 iff err4 < err6.  Elements 2j, 2j+1 share a packed register; the two
+// candidates' trees run side by side from level 2 on.
 // ---------------------------------------------------------------------------------------------
-struct Fwd46Candidate {
-    uint32_t codes[2];
-    uint32_t scale;
-    float err;
+struct Fwd46Scale {
+    uint32_t code;
+    float d;
+    uint64_t rr;       // (1/d, 1/d)
 };
 
-// Candidate with grid maximum k: s = RNE_E4M3(a/(g*k)), d = s*g, codes = RNE_E2M1(x*(1/d)),
-// err = tree sum of (x - val*d)^2.  A zero scale gives sign-preserving zero codes (x*0) and
-// err = sum x^2.
-__device__ __forceinline__ Fwd46Candidate fwd46_candidate(const float (&x)[16], float a, float g, float k) {
-    Fwd46Candidate c;
-    const float t = __fdiv_rn(a, __fmul_rn(g, k));
-    c.scale = e4m3_rne(t);
-    const float d = __fmul_rn(e4m3_value(c.scale), g);
-    const float r = (c.scale == 0) ? 0.0f : __frcp_rn(d);
-    float sq[16];
+__device__ __forceinline__ Fwd46Scale fwd46_scale(float a, float g, float gk) {
+    Fwd46Scale c;
+    c.code = e4m3_rne(__fdiv_rn(a, gk));
+    const float d = __fmul_rn(e4m3_value(c.code), g);
+    const float r = (c.code == 0) ? 0.0f : __frcp_rn(d);
+    c.rr = f2(r, r);
+    c.d = d;
+    return c;
+}
+
+// Codes of one candidate (two words: elements 0..7, 8..15) and its 8 level-1 error sums
+// (element pairs 2j, 2j+1).
+__device__ __forceinline__ void fwd46_candidate(const uint64_t (&X)[8], const Fwd46Scale &sc, uint32_t (&codes)[2],
+                                                float (&e1)[8]) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         float q[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(x[8 * h + i], r);
-        c.codes[h] = e2m1x8(q);
+        for (int i = 0; i < 4; ++i) f2_split(f2_mul(X[4 * h + i], sc.rr), q[2 * i], q[2 * i + 1]);
+        codes[h] = e2m1x8(q);
         float val[8];
-        e2m1x8_values(c.codes[h], val);
+        e2m1x8_values(codes[h], val);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float e = __fsub_rn(x[8 * h + i], __fmul_rn(val[i], d));
-            sq[8 * h + i] = __fmul_rn(e, e);
+        for (int i = 0; i < 4; ++i) {
+            // x - val*d in scalar mul.rn/sub.rn, which are never fused: a packed multiply feeding a
+            // packed subtract may be contracted into one fused multiply-add
+            float x0, x1;
+            f2_split(X[4 * h + i], x0, x1);
+            const float e0 = __fsub_rn(x0, __fmul_rn(val[2 * i], sc.d));
+            const float e1v = __fsub_rn(x1, __fmul_rn(val[2 * i + 1], sc.d));
+            float s0, s1;
+            f2_split(f2_mul(f2(e0, e1v), f2(e0, e1v)), s0, s1);
+            e1[4 * h + i] = __fadd_rn(s0, s1);
         }
     }
-    c.err = tree_sum<16>(sq);
-    return c;
 }
 
 __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
@@ -113,6 +154,7 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
     const float A = __uint_as_float(*amax_word);
     const bool zero_tensor = !(A >= kTiny);
     const float g = zero_tensor ? 1.0f : __fdiv_rn(A, kFwd46Denominator);
+    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
 
     const uint32_t G = (uint32_t)(C >> 4);                 // groups per row (a multiple of 8)
@@ -125,193 +167,54 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
         const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (uint64_t)q * 16);
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        float xv[16];
-        float a = 0.0f;
+        uint64_t X[8];
+        float m8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            xv[2 * i] = bf16_lo(w[i]);
-            xv[2 * i + 1] = bf16_hi(w[i]);
-            a = fmaxf(a, fmaxf(fabsf(xv[2 * i]), fabsf(xv[2 * i + 1])));
+            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+            X[i] = f2(lo, hi);
+            m8[i] = fmaxf(fabsf(lo), fabsf(hi));
         }
-        const Fwd46Candidate c6 = fwd46_candidate(xv, a, g, 6.0f);
-        const Fwd46Candidate c4 = fwd46_candidate(xv, a, g, 4.0f);
-        const bool pick4 = c4.err < c6.err;                 // a tie keeps the full grid
-        const uint32_t code0 = pick4 ? c4.codes[0] : c6.codes[0];
-        const uint32_t code1 = pick4 ? c4.codes[1] : c6.codes[1];
-        const uint32_t s = pick4 ? c4.scale : c6.scale;
+#pragma unroll
+        for (int s = 8; s > 1; s >>= 1) {
+#pragma unroll
+            for (int i = 0; i < s / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
+        }
+        const float a = m8[0];
+        const Fwd46Scale s6 = fwd46_scale(a, g, g6), s4 = fwd46_scale(a, g, g4);
+        uint32_t c6[2], c4[2];
+        float e6[8], e4[8];
+        fwd46_candidate(X, s6, c6, e6);
+        fwd46_candidate(X, s4, c4, e4);
+        uint64_t t[8];   // (candidate 6, candidate 4) level-1 sums, then levels 2..4 together
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
+#pragma unroll
+        for (int s = 8; s > 1; s >>= 1) {
+#pragma unroll
+            for (int i = 0; i < s / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
+        }
+        float err6, err4;
+        f2_split(t[0], err6, err4);
+        const bool pick4 = err4 < err6;                    // a tie keeps the full grid
+        const uint32_t code0 = pick4 ? c4[0] : c6[0];
+        const uint32_t code1 = pick4 ? c4[1] : c6[1];
+        const uint32_t sc = pick4 ? s4.code : s6.code;
         *reinterpret_cast<uint2 *>(codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8) = make_uint2(code0, code1);
         // four consecutive groups (same row, q % 4 == 0 .. 3) share one scale word
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, s, 1);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, s, 2);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, s, 3);
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if ((lane & 3) == 0)
-            *reinterpret_cast<uint32_t *>(scales + sf_offset((int64_t)r, q, C)) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            *reinterpret_cast<uint32_t *>(scales + sf_offset((int64_t)r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
 }
 
 // ---------------------------------------------------------------------------------------------
-// MS-EDEN producer ([QII-tg] "Method"; [QII-th] "Question 1"; [FAF]: both layouts in one pass).
-// One CTA of 128 threads per 128x128 tile, loaded once by TMA (128-byte swizzle, two boxes of
-// 64 columns).  Row view: thread t rotates and quantizes row t of the tile (a 128-block along
-// the columns).  Column view: thread t does column t (a 128-block along the rows), giving row
-// t of the transposed view.  Per 128-block: y = H D x, per group p = max|y|/6 and codes =
-// RNE_E2M1(y * (1/p)), per block S = sum y^2 / sum p * <val, y>; the pre-scale S*p goes to
-// the workspace (fp32, scale-factor order) and the view max |y| to an atomicMax word.
+// The 128 rotation signs of one backward call: bit i of Philox(seed, tensor id 0) word i/32 set
+// -> negate element i of every 128-block ([QII-th] "Question 1": one shared rotation and seed).
 // ---------------------------------------------------------------------------------------------
-
-// Unnormalised Walsh-Hadamard butterfly, strides 1..64, (a+b, a-b) with a at the lower index.
-__device__ __forceinline__ void fwht128(float (&y)[128]) {
-#pragma unroll
-    for (int h = 1; h < 128; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-            if ((i & h) == 0) {
-                const float a = y[i], b = y[i + h];
-                y[i] = __fadd_rn(a, b);
-                y[i + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-}
-
-// Quantize one rotated 128-block: 16 code words (element 8w+i in nibble i of word w), 8 pre-scales.
-__device__ __forceinline__ void msed_block(float (&y)[128], uint32_t (&cw)[16], float (&P)[8], float &amax) {
-    float nq[8], ptq[8], pq[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        float a = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(y[16 * q + i]));
-        amax = fmaxf(amax, a);
-        const bool live = a >= kTiny;
-        const float p = live ? __fdiv_rn(a, 6.0f) : 0.0f;
-        const float r = live ? __frcp_rn(p) : 0.0f;          // flushed group: sign-preserving zeros
-        float tv[16], nv[16];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(y[16 * q + 8 * h + i], r);
-            cw[2 * q + h] = e2m1x8(v);
-            float val[8];
-            e2m1x8_values(cw[2 * q + h], val);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float yi = y[16 * q + 8 * h + i];
-                tv[8 * h + i] = __fmul_rn(val[i], yi);
-                nv[8 * h + i] = __fmul_rn(yi, yi);
-            }
-        }
-        pq[q] = p;
-        nq[q] = live ? tree_sum<16>(nv) : 0.0f;
-        ptq[q] = live ? __fmul_rn(p, tree_sum<16>(tv)) : 0.0f;
-    }
-    const float num = tree_sum<8>(nq), den = tree_sum<8>(ptq);
-    const float S = den > 0.0f ? __fdiv_rn(num, den) : 1.0f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) P[q] = __fmul_rn(S, pq[q]);
-}
-
-// The 128 rotation signs: bit i of Philox(seed, tensor id 0) word i/32 set -> negate element i.
 __device__ __forceinline__ uint4 rotation_sign_words(uint64_t seed) { return philox_block(seed, 0u, 0ull); }
-
-__device__ __forceinline__ uint32_t sign_bit(const uint4 &sw, int i) {
-    const uint32_t w = (i < 32) ? sw.x : (i < 64) ? sw.y : (i < 96) ? sw.z : sw.w;
-    return ((w >> (i & 31)) & 1u) << 31;
-}
-
-__device__ __forceinline__ void store_block(uint8_t *codes_dst, float *P_base, int64_t vr, int64_t j0, int64_t VC,
-                                            const uint32_t (&cw)[16], const float (&P)[8]) {
-    uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
-    *reinterpret_cast<float4 *>(P_base + sf_offset(vr, j0, VC)) = make_float4(P[0], P[1], P[2], P[3]);
-    *reinterpret_cast<float4 *>(P_base + sf_offset(vr, j0 + 4, VC)) = make_float4(P[4], P[5], P[6], P[7]);
-}
-
-template <bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(128) msed_tile_kernel(const __grid_constant__ CUtensorMap tmap, int64_t R, int64_t C,
-                                                        uint64_t seed, uint8_t *__restrict__ row_codes,
-                                                        float *__restrict__ row_P, uint32_t *__restrict__ row_amax,
-                                                        uint8_t *__restrict__ col_codes, float *__restrict__ col_P,
-                                                        uint32_t *__restrict__ col_amax) {
-    extern __shared__ __align__(1024) uint8_t smem_dyn[];
-    uint8_t *tile = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ uint32_t red[2][4];
-
-    const int t = threadIdx.x;
-    const int64_t c0 = (int64_t)blockIdx.x * 128, r0 = (int64_t)blockIdx.y * 128;
-    const uint32_t bar_a = smem_u32(&bar);
-    if (t == 0) {
-        prefetch_tmap(&tmap);
-        mbar_init(bar_a, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (t == 0) {
-        mbar_arrive_expect_tx(bar_a, 128 * 128 * 2);
-        tma_load_2d(smem_u32(tile), &tmap, (int32_t)c0, (int32_t)r0, bar_a);
-        tma_load_2d(smem_u32(tile + 16384), &tmap, (int32_t)(c0 + 64), (int32_t)r0, bar_a);
-    }
-    const uint4 sw = rotation_sign_words(seed);
-    const bool ok = mbar_wait(bar_a, 0);
-
-    float amax_r = 0.0f, amax_c = 0.0f;
-    if (ok && DO_ROW) {
-        // row t: 16 chunks of 8 bf16; chunk c of box h sits at chunk position c ^ (t & 7)
-        float y[128];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(tile + h * 16384 + t * 128 + ((c ^ (t & 7)) << 4));
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int e = 64 * h + 8 * c + 2 * i;
-                    y[e] = __uint_as_float(__float_as_uint(bf16_lo(w[i])) ^ sign_bit(sw, e));
-                    y[e + 1] = __uint_as_float(__float_as_uint(bf16_hi(w[i])) ^ sign_bit(sw, e + 1));
-                }
-            }
-        }
-        fwht128(y);
-        uint32_t cw[16];
-        float P[8];
-        msed_block(y, cw, P, amax_r);
-        const int64_t vr = r0 + t;
-        store_block(row_codes + vr * (C >> 1) + (c0 >> 1), row_P, vr, c0 >> 4, C, cw, P);
-    }
-    if (ok && DO_COL) {
-        // column t: element i is row i of the tile
-        const int h = t >> 6, cc = t & 63;
-        const uint8_t *base = tile + h * 16384 + ((cc & 7) << 1);
-        float y[128];
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-            const uint16_t b = *reinterpret_cast<const uint16_t *>(base + i * 128 + ((((cc >> 3) ^ (i & 7))) << 4));
-            y[i] = __uint_as_float((((uint32_t)b) << 16) ^ sign_bit(sw, i));
-        }
-        fwht128(y);
-        uint32_t cw[16];
-        float P[8];
-        msed_block(y, cw, P, amax_c);
-        const int64_t vr = c0 + t;                 // row of the transposed view [C][R]
-        store_block(col_codes + vr * (R >> 1) + (r0 >> 1), col_P, vr, r0 >> 4, R, cw, P);
-    }
-    // view maxima: warp reduce, then one atomicMax per CTA
-    const uint32_t br = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_r));
-    const uint32_t bc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_c));
-    if ((t & 31) == 0) {
-        red[0][t >> 5] = br;
-        red[1][t >> 5] = bc;
-    }
-    __syncthreads();
-    if (t == 0) {
-        if (DO_ROW) atomicMax(row_amax, max(max(red[0][0], red[0][1]), max(red[0][2], red[0][3])));
-        if (DO_COL) atomicMax(col_amax, max(max(red[1][0], red[1][1]), max(red[1][2], red[1][3])));
-    }
-}
 
 // ---------------------------------------------------------------------------------------------
 // MS-EDEN scale finalize: group scale = SR_E4M3(S*p*(1/g)) with g = A/1536 ([QII-tg] "Method":

@@ -50,7 +50,10 @@ def _x(R, C, seed, scale=1.0):
 # (M, N, K): single tile, N % 256 != 0 (128-wide tiles), K not a multiple of 256 (half stage),
 # several stages around the ring, a long K.
 SHAPES = [(128, 128, 128), (128, 256, 256), (256, 256, 256), (384, 640, 1152), (256, 512, 2048), (128, 384, 4224),
-          (256, 256, 8192)]
+          (256, 256, 8192),
+          # M and N multiples of 256 run on SM pairs: several tiles each way, a K tail (4224 = 16.5 x 256),
+          # and more tiles (16 x 16) than resident pairs, so each pair loops over tiles
+          (512, 768, 1024), (768, 512, 4224), (4096, 4096, 512)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -62,7 +65,7 @@ def test_gemm_forward_operands(M, N, K, dtype):
     check(got, va, vb, 1.0, bf16=dtype == qt2.QT2_DTYPE_BF16)
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (384, 640, 1152), (128, 384, 4224)])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (384, 640, 1152), (128, 384, 4224), (512, 1024, 2048)])
 def test_gemm_msedEN_operands(M, N, K):
     seed = 5
     va = O.msedEN(_x(M, K, 3, 1e-4), seed, 1, "row")
