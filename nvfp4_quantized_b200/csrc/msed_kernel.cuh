@@ -13,26 +13,71 @@
 // S = sum y^2 / sum p * <val, y>; the pre-scale S*p is written (fp32, tensor-core scale order)
 // for the finalize pass and the view max |y| merged with atomicMax.  Every floating-point
 // step is one IEEE binary32 operation rounded to nearest-even in the reference order; the packed
-// f32x2 forms below are two such operations side by side.
+// f32x2 forms below are two such operations side by side, and an FMA whose product is an exact
+// +-1 multiple is one rounded addition or subtraction.
 //
-// Design: persistent CTAs of 256 threads; each thread rotates and quantizes one 128-element
-// vector per tile entirely in registers (64 packed fp32 pairs).  Tiles stream in by TMA
-// (128-byte swizzle, two-deep ring) while the previous one is processed:
-//   both views : 128x128 tiles, threads 0..127 take rows, 128..255 take columns;
-//   rows only  : 256x128 tiles (128x128 when rows % 256 != 0), one row per thread;
-//   columns only: 128x256 tiles (128x128 when cols % 256 != 0), one column per thread.
+// Design: persistent CTAs of 512 threads (16 warps at up to 128 registers, so an SM keeps 16
+// warps in flight), 128x128 bf16 tiles streamed by TMA (128-byte swizzle) through a 3-deep ring.
+// Two threads (adjacent lanes, h = 0, 1) share one 128-element vector: thread h holds elements
+// [64h, 64h + 64) as 32 packed pairs and runs the butterfly strides 1..32 in registers; stride 64
+// crosses the pair with one shuffle per packed value.  After it, thread h owns the 16-groups
+// {2h, 2h+1} and {4+2h, 5+2h} of the block and quantizes them; the block sums for S meet
+// through two more shuffles.  To make the cross step the same instructions on both threads,
+// thread 1 keeps its half with the two 32-element quarters swapped (natural pair n of its half
+// sits in slot (n + 16) % 32); that turns its stride-32 and stride-64 subtractions around, and
+// an FMA with sigma = +-1 gives each thread its own operand order exactly (signed zeros included).
+//   both views : warps 0..7 take the rows of each tile, warps 8..15 its columns;
+//   one view   : warps 0..7 and 8..15 take alternate tiles.
+// A ring stage is refilled by the last warp that has read it (a shared counter), so the two
+// halves of the CTA drift freely by up to the ring depth.
 #pragma once
 
 #include "quant_kernels.cuh"
 
 namespace qt2 {
 
-// Butterfly stages with strides 2..64 on P[j] = (y[2j], y[2j+1]) (stride 1 is done on input).
-__device__ __forceinline__ void fwht_packed_tail(uint64_t (&P)[64]) {
+struct MsedCfg {
+    static constexpr int kThreads = 512;
+    static constexpr int kTeamWarps = 8;
+    static constexpr int kStages = 3;
+    static constexpr int kTileBytes = 128 * 128 * 2;
+    static constexpr int kSmemBytes = kStages * kTileBytes + 1024;
+};
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t shfl_xor1_u64(uint64_t v) {
+    uint32_t lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+    lo = __shfl_xor_sync(0xFFFFFFFFu, lo, 1);
+    hi = __shfl_xor_sync(0xFFFFFFFFu, hi, 1);
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
+// Byte offset of tile element (r, c) in a 128x128 tile held as two 128x64 boxes (128-byte swizzle).
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+    return (uint32_t)((c >> 6) * 16384 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+}
+
+// Butterfly strides 2..64 and quantization of one vector held by a thread pair.
+// In: P = the thread's half after stride 1, in slot order; sg = (sigma, sigma), nsg = -sg with
+// sigma = +1 on thread 0 and -1 on thread 1.
+// Out: cw[2g], cw[2g+1] = codes of local group g (element 8w+i of the group in nibble i of
+// word w); Pq[g] = S * p of local group g.  Local groups 0, 1, 2, 3 are the block's groups 2h,
+// 2h+1, 4+2h, 5+2h.  amax = running max |y|.
+__device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint64_t nsg, uint32_t (&cw)[8],
+                                            float (&Pq)[4], float &amax) {
+    // strides 2, 4, 8, 16: slots j and j + hp of the same 16-slot half, same order on both threads
 #pragma unroll
-    for (int hp = 1; hp < 64; hp <<= 1) {
+    for (int hp = 1; hp < 16; hp <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < 32; ++j) {
             if ((j & hp) == 0) {
                 const uint64_t a = P[j], b = P[j + hp];
                 P[j] = f2_add(a, b);
@@ -40,18 +85,29 @@ __device__ __forceinline__ void fwht_packed_tail(uint64_t (&P)[64]) {
             }
         }
     }
-}
-
-// Quantize one rotated 128-block held as packed pairs: 16 code words (element 8w+i in nibble i
-// of word w), 8 pre-scales S*p, running max of |y|.
-__device__ __forceinline__ void msed_quantize_packed(const uint64_t (&P)[64], uint32_t (&cw)[16], float (&Pq)[8],
-                                                     float &amax) {
-    float nq[8], ptq[8], pq[8];
+    // stride 32: thread 0 forms (u + v, u - v), thread 1 (its halves swapped) (v - u, v + u)
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int j = 0; j < 16; ++j) {
+        const uint64_t u = P[j], v = P[j + 16];
+        P[j] = f2_fma(sg, u, v);
+        P[j + 16] = f2_fma(nsg, v, u);
+    }
+    // stride 64 across the pair: both threads send slot 16 + k and keep slot k.  Thread 0 keeps
+    // z[2k] and receives z[64 + 2k]; thread 1 keeps z[96 + 2k] and receives z[32 + 2k].
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const uint64_t recv = shfl_xor1_u64(P[16 + k]);
+        const uint64_t keep = P[k];
+        P[k] = f2_add(keep, recv);                        // y[i] = z[i] + z[i + 64]
+        P[16 + k] = f2_fma(sg, keep, f2_mul(recv, nsg));  // y[i + 64] = z[i] - z[i + 64]
+    }
+
+    float nq[4], ptq[4], pq[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
         float y[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f2_split(P[8 * q + i], y[2 * i], y[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) f2_split(P[8 * g + i], y[2 * i], y[2 * i + 1]);
         float m8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1]));
@@ -68,18 +124,18 @@ __device__ __forceinline__ void msed_quantize_packed(const uint64_t (&P)[64], ui
         const uint64_t rr = f2(r, r);
         float v[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f2_split(f2_mul(P[8 * q + i], rr), v[2 * i], v[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) f2_split(f2_mul(P[8 * g + i], rr), v[2 * i], v[2 * i + 1]);
         float val[16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int hh = 0; hh < 2; ++hh) {
             float vh[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) vh[i] = v[8 * h + i];
-            cw[2 * q + h] = e2m1x8(vh);
+            for (int i = 0; i < 8; ++i) vh[i] = v[8 * hh + i];
+            cw[2 * g + hh] = e2m1x8(vh);
             float dv[8];
-            e2m1x8_values(cw[2 * q + h], dv);
+            e2m1x8_values(cw[2 * g + hh], dv);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) val[8 * h + i] = dv[i];
+            for (int i = 0; i < 8; ++i) val[8 * hh + i] = dv[i];
         }
         // products val*y and y*y, then the 16-term trees; level 1 pairs adjacent elements,
         // levels 2..4 run on (t, n) packed together
@@ -87,8 +143,8 @@ __device__ __forceinline__ void msed_quantize_packed(const uint64_t (&P)[64], ui
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float t0, t1, n0, n1;
-            f2_split(f2_mul(f2(val[2 * i], val[2 * i + 1]), P[8 * q + i]), t0, t1);
-            f2_split(f2_mul(P[8 * q + i], P[8 * q + i]), n0, n1);
+            f2_split(f2_mul(f2(val[2 * i], val[2 * i + 1]), P[8 * g + i]), t0, t1);
+            f2_split(f2_mul(P[8 * g + i], P[8 * g + i]), n0, n1);
             tn[i] = f2(__fadd_rn(t0, t1), __fadd_rn(n0, n1));
         }
 #pragma unroll
@@ -98,170 +154,157 @@ __device__ __forceinline__ void msed_quantize_packed(const uint64_t (&P)[64], ui
         }
         float tg, ng;
         f2_split(tn[0], tg, ng);
-        pq[q] = p;
-        nq[q] = live ? ng : 0.0f;
-        ptq[q] = live ? __fmul_rn(p, tg) : 0.0f;
+        pq[g] = p;
+        nq[g] = live ? ng : 0.0f;
+        ptq[g] = live ? __fmul_rn(p, tg) : 0.0f;
     }
-    const float num = tree_sum<8>(nq), den = tree_sum<8>(ptq);
+    // Block sums over the 8 groups as the balanced tree ((G0+G1)+(G2+G3)) + ((G4+G5)+(G6+G7)):
+    // this thread's level-1 sums are (G2h + G2h+1) and (G4+2h + G5+2h); level 2 adds the
+    // partner's (addition commutes, so both threads get the same bits).
+    const uint64_t lv_a = f2(__fadd_rn(nq[0], nq[1]), __fadd_rn(ptq[0], ptq[1]));
+    const uint64_t lv_b = f2(__fadd_rn(nq[2], nq[3]), __fadd_rn(ptq[2], ptq[3]));
+    const uint64_t lo = f2_add(lv_a, shfl_xor1_u64(lv_a)), hi = f2_add(lv_b, shfl_xor1_u64(lv_b));
+    float num, den;
+    f2_split(f2_add(lo, hi), num, den);
     const float S = den > 0.0f ? __fdiv_rn(num, den) : 1.0f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) Pq[q] = __fmul_rn(S, pq[q]);
+    for (int g = 0; g < 4; ++g) Pq[g] = __fmul_rn(S, pq[g]);
 }
 
-__device__ __forceinline__ void msed_store(uint8_t *codes_dst, float *P_base, int64_t vr, int64_t j0, int64_t VC,
-                                           const uint32_t (&cw)[16], const float (&P)[8]) {
-    uint4 *dst = reinterpret_cast<uint4 *>(codes_dst);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
-    *reinterpret_cast<float4 *>(P_base + sf_offset(vr, j0, VC)) = make_float4(P[0], P[1], P[2], P[3]);
-    *reinterpret_cast<float4 *>(P_base + sf_offset(vr, j0 + 4, VC)) = make_float4(P[4], P[5], P[6], P[7]);
+// Codes of the thread's groups {2h, 2h+1} and {4+2h, 5+2h} of a 128-block starting at group j0
+// of view row vr (codes_row points at the block's first code byte); pre-scales in tensor-core
+// scale order.
+__device__ __forceinline__ void msed_store(uint8_t *codes_row, float *P_base, int64_t vr, int64_t j0, int64_t VC,
+                                           int h, const uint32_t (&cw)[8], const float (&Pq)[4]) {
+    *reinterpret_cast<uint4 *>(codes_row + 16 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    *reinterpret_cast<uint4 *>(codes_row + 32 + 16 * h) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    *reinterpret_cast<float2 *>(P_base + sf_offset(vr, j0 + 2 * h, VC)) = make_float2(Pq[0], Pq[1]);
+    *reinterpret_cast<float2 *>(P_base + sf_offset(vr, j0 + 4 + 2 * h, VC)) = make_float2(Pq[2], Pq[3]);
 }
 
-// Byte offset of tile element (r, c) in a buffer of 128x64 boxes loaded with the 128-byte swizzle.
-template <int TC>
-__device__ __forceinline__ uint32_t tile_off(int r, int c) {
-    const int box = (r >> 7) * (TC / 64) + (c >> 6), rr = r & 127;
-    return (uint32_t)(box * 16384 + rr * 128 + ((((c & 63) >> 3) ^ (rr & 7)) << 4) + ((c & 7) << 1));
-}
-
-template <int TR, int TC, bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, 1)
+template <bool DO_ROW, bool DO_COL>
+__global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     msed_kernel(const __grid_constant__ CUtensorMap tmap, int64_t R, int64_t C, uint64_t seed,
                 uint8_t *__restrict__ row_codes, float *__restrict__ row_P, uint32_t *__restrict__ row_amax,
                 uint8_t *__restrict__ col_codes, float *__restrict__ col_P, uint32_t *__restrict__ col_amax) {
-    constexpr int kTileBytes = TR * TC * 2;
-    constexpr int kBoxes = (TR / 128) * (TC / 64);
+    using Cfg = MsedCfg;
+    constexpr int NS = Cfg::kStages;
+    constexpr bool kBoth = DO_ROW && DO_COL;
+    constexpr uint32_t kConsumers = kBoth ? 2 * Cfg::kTeamWarps : Cfg::kTeamWarps;   // warps reading a tile
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t *buf0 = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t bar[2];
-    __shared__ uint32_t pair_mask[64];   // row view: sign bits of elements 2j, 2j+1 at bits 15 and 31
-    __shared__ uint32_t elem_mask[128];  // column view: sign bit of element i at bit 31
-    __shared__ uint32_t red[2][8];
+    __shared__ __align__(8) uint64_t bar[NS];
+    __shared__ uint32_t done_cnt[NS];           // warps done reading the stage, summed over its rounds
+    __shared__ int last_issued[NS];             // local index of the last tile loaded into the stage
+    __shared__ __align__(16) uint2 sgn2[64];    // sign flips of elements 2n, 2n+1 at bit 31 of .x, .y
 
-    const int t = threadIdx.x;
-    const int64_t tiles_c = C / TC, ntiles = (R / TR) * tiles_c;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int team = warp >= Cfg::kTeamWarps ? 1 : 0;
+    const int h = lane & 1;
+    const int64_t tiles_c = C >> 7, ntiles = (R >> 7) * tiles_c;
+    const int64_t my_tiles = ntiles > (int64_t)blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     const uint32_t bar0 = smem_u32(&bar[0]);
+
+    auto issue = [&](int64_t i) {   // local tile i into stage i % NS
+        const int64_t tile = blockIdx.x + i * (int64_t)gridDim.x;
+        const int32_t r0 = (int32_t)((tile / tiles_c) << 7), c0 = (int32_t)((tile % tiles_c) << 7);
+        const int s = (int)(i % NS);
+        const uint32_t fb = bar0 + 8 * s;
+        last_issued[s] = (int)i;
+        mbar_arrive_expect_tx(fb, Cfg::kTileBytes);
+        tma_load_2d(smem_u32(buf0 + s * Cfg::kTileBytes), &tmap, c0, r0, fb);
+        tma_load_2d(smem_u32(buf0 + s * Cfg::kTileBytes + 16384), &tmap, c0 + 64, r0, fb);
+    };
     if (t == 0) {
         prefetch_tmap(&tmap);
-        mbar_init(bar0, 1);
-        mbar_init(bar0 + 8, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar0 + 8 * s, 1);
+            done_cnt[s] = 0;
+            last_issued[s] = -1;
+        }
         fence_mbar_init();
     }
-    {
+    if (t < 64) {
         const uint4 sw = rotation_sign_words(seed);   // bit i of the 128 signs: element i negated
         const uint32_t w[4] = {sw.x, sw.y, sw.z, sw.w};
-        if (t < 128) elem_mask[t] = ((w[t >> 5] >> (t & 31)) & 1u) << 31;
-        if (t < 64) {
-            const int e = 2 * t;
-            pair_mask[t] = (((w[e >> 5] >> (e & 31)) & 1u) << 15) | (((w[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) << 31);
-        }
+        const int e = 2 * t;
+        sgn2[t] = make_uint2(((w[e >> 5] >> (e & 31)) & 1u) << 31, ((w[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) << 31);
     }
     __syncthreads();
+    if (t == 0)
+        for (int64_t i = 0; i < NS && i < my_tiles; ++i) issue(i);
 
-    auto issue = [&](int64_t tile, int b) {
-        const int32_t r0 = (int32_t)((tile / tiles_c) * TR), c0 = (int32_t)((tile % tiles_c) * TC);
-        const uint32_t fb = bar0 + 8 * b;
-        mbar_arrive_expect_tx(fb, kTileBytes);
+    const float sigma = h ? -1.0f : 1.0f;
+    const uint64_t sg = f2(sigma, sigma), nsg = f2(-sigma, -sigma);
+    const bool rows = kBoth ? team == 0 : DO_ROW;
+    const int u = (t & (Cfg::kTeamWarps * 32 - 1)) >> 1;   // the pair's row (or column) of the tile
+    float amax = 0.0f;
+    const int64_t i0 = kBoth ? 0 : team, step = kBoth ? 1 : 2;
+    for (int64_t i = i0; i < my_tiles; i += step) {
+        const int s = (int)(i % NS);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, (uint32_t)((i / NS) & 1)))) break;   // warp-uniform
+        const uint8_t *tb = buf0 + s * Cfg::kTileBytes;
+        const int64_t tile = blockIdx.x + i * (int64_t)gridDim.x;
+        const int64_t r0 = (tile / tiles_c) << 7, c0 = (tile % tiles_c) << 7;
+        uint64_t P[32];
+        if (rows) {
+            // row u, elements [64h, 64h + 64); register chunk c holds element chunk 8h + ((c + 4h) & 7)
 #pragma unroll
-        for (int br = 0; br < TR / 128; ++br)
+            for (int c = 0; c < 8; ++c) {
+                const int e = 8 * h + ((c + 4 * h) & 7);
+                const uint4 v = *reinterpret_cast<const uint4 *>(tb + tile_off(u, 8 * e));
+                const uint4 m01 = *reinterpret_cast<const uint4 *>(&sgn2[4 * e]);
+                const uint4 m23 = *reinterpret_cast<const uint4 *>(&sgn2[4 * e + 2]);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                const uint32_t ml[4] = {m01.x, m01.z, m23.x, m23.z}, mh[4] = {m01.y, m01.w, m23.y, m23.w};
 #pragma unroll
-            for (int bc = 0; bc < TC / 64; ++bc)
-                tma_load_2d(smem_u32(buf0 + b * kTileBytes + (br * (TC / 64) + bc) * 16384), &tmap, c0 + 64 * bc,
-                            r0 + 128 * br, fb);
-    };
-    int issued = 0;
-    if (t == 0) {
-        for (int b = 0; b < 2; ++b) {
-            const int64_t tile = blockIdx.x + (int64_t)b * gridDim.x;
-            if (tile < ntiles) {
-                issue(tile, b);
-                issued = b + 1;
-            }
-        }
-    }
-    (void)kBoxes;
-
-    float amax_r = 0.0f, amax_c = 0.0f;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-        const int b = i & 1;
-        const bool ok = mbar_wait(bar0 + 8 * b, (i >> 1) & 1);
-        if (__syncthreads_or(!ok)) break;
-        const uint8_t *tb = buf0 + b * kTileBytes;
-        const int64_t r0 = (tile / tiles_c) * TR, c0 = (tile % tiles_c) * TC;
-        const bool row_thread = DO_ROW && (DO_COL ? t < 128 : t < TR);
-        const bool col_thread = DO_COL && (DO_ROW ? t >= 128 : t < TC);
-        if (row_thread || col_thread) {
-            // Only the loads and the stores differ between a row vector and a column vector; the
-            // rotation and quantization below are one code path for both (instruction-cache reuse).
-            uint64_t P[64];
-            if (row_thread) {
-                const int rr = t;   // row of the tile; its 128-block is the whole tile width (TC = 128)
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(tb + tile_off<TC>(rr, 8 * c));
-                    const uint4 m = *reinterpret_cast<const uint4 *>(&pair_mask[4 * c]);
-                    const uint32_t w[4] = {v.x ^ m.x, v.y ^ m.y, v.z ^ m.z, v.w ^ m.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float x0 = bf16_lo(w[k]), x1 = bf16_hi(w[k]);
-                        P[4 * c + k] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
-                    }
-                }
-            } else {
-                const int cc = DO_ROW ? t - 128 : t;   // column of the tile; its 128-block is rows 0..127
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const uint32_t u0 = *reinterpret_cast<const uint16_t *>(tb + tile_off<TC>(2 * j, cc));
-                    const uint32_t u1 = *reinterpret_cast<const uint16_t *>(tb + tile_off<TC>(2 * j + 1, cc));
-                    const float x0 = __uint_as_float((u0 << 16) ^ elem_mask[2 * j]);
-                    const float x1 = __uint_as_float((u1 << 16) ^ elem_mask[2 * j + 1]);
-                    P[j] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
+                for (int k = 0; k < 4; ++k) {
+                    const float x0 = __uint_as_float((w[k] << 16) + ml[k]);   // adding 2^31 flips the sign bit
+                    const float x1 = __uint_as_float((w[k] & 0xFFFF0000u) ^ mh[k]);
+                    P[4 * c + k] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
                 }
             }
-            fwht_packed_tail(P);
-            uint32_t cw[16];
-            float Pq[8];
-            float vmax = 0.0f;
-            msed_quantize_packed(P, cw, Pq, vmax);
-            if (row_thread) {
-                amax_r = fmaxf(amax_r, vmax);
-                const int64_t vr = r0 + t;
-                msed_store(row_codes + vr * (C >> 1) + (c0 >> 1), row_P, vr, c0 >> 4, C, cw, Pq);
-            } else {
-                amax_c = fmaxf(amax_c, vmax);
-                const int64_t vr = c0 + (DO_ROW ? t - 128 : t);   // row of the transposed view [C][R]
-                msed_store(col_codes + vr * (R >> 1) + (r0 >> 1), col_P, vr, r0 >> 4, R, cw, Pq);
+        } else {
+            // column u, rows [64h, 64h + 64); slot j holds rows 2n, 2n + 1 of the half, n = (j + 16h) % 32
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const int n = (j + 16 * h) & 31, rr = 64 * h + 2 * n;
+                const uint4 m = *reinterpret_cast<const uint4 *>(&sgn2[rr >> 1]);
+                const uint32_t u0 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr, u));
+                const uint32_t u1 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 1, u));
+                const uint32_t u2 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 2, u));
+                const uint32_t u3 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 3, u));
+                const float x0 = __uint_as_float((u0 << 16) + m.x), x1 = __uint_as_float((u1 << 16) + m.y);
+                const float x2 = __uint_as_float((u2 << 16) + m.z), x3 = __uint_as_float((u3 << 16) + m.w);
+                P[j] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
+                P[j + 1] = f2(__fadd_rn(x2, x3), __fsub_rn(x2, x3));
             }
         }
-        __syncthreads();   // every thread is done with this buffer
-        if (t == 0) {
-            const int64_t next = tile + 2 * (int64_t)gridDim.x;
-            if (next < ntiles) {
-                issue(next, b);
-                issued = i + 3;
-            }
+        // The tile is in registers: release the stage; the last warp to do so refills it.
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            const uint32_t old = atomicAdd(&done_cnt[s], 1u);
+            if (old == (uint32_t)(i / NS + 1) * kConsumers - 1 && i + NS < my_tiles) issue(i + NS);
+        }
+        uint32_t cw[8];
+        float Pq[4];
+        msed_vector(P, sg, nsg, cw, Pq, amax);
+        if (rows) {
+            const int64_t vr = r0 + u;
+            msed_store(row_codes + vr * (C >> 1) + (c0 >> 1), row_P, vr, c0 >> 4, C, h, cw, Pq);
+        } else {
+            const int64_t vr = c0 + u;   // row of the transposed view [C][R]
+            msed_store(col_codes + vr * (R >> 1) + (r0 >> 1), col_P, vr, r0 >> 4, R, h, cw, Pq);
         }
     }
-    if (t == 0) {
-        // Only after a timeout can loads still be in flight: wait (bounded) for them.
-        for (int k = i; k < issued; ++k) mbar_wait(bar0 + 8 * (k & 1), (k >> 1) & 1);
-    }
-    const uint32_t br = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_r));
-    const uint32_t bc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax_c));
-    if ((t & 31) == 0) {
-        red[0][t >> 5] = br;
-        red[1][t >> 5] = bc;
-    }
+    const uint32_t bm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
+    if (lane == 0 && bm != 0) atomicMax(rows ? row_amax : col_amax, bm);
     __syncthreads();
     if (t == 0) {
-        uint32_t mr = 0, mc = 0;
-        for (int k = 0; k < 8; ++k) {
-            mr = max(mr, red[0][k]);
-            mc = max(mc, red[1][k]);
-        }
-        if (DO_ROW) atomicMax(row_amax, mr);
-        if (DO_COL) atomicMax(col_amax, mc);
+        // Only after a timeout can a load still be in flight: wait (bounded) for each stage's last one.
+        for (int s = 0; s < NS; ++s)
+            if (last_issued[s] >= 0) mbar_wait(bar0 + 8 * s, (uint32_t)((last_issued[s] / NS) & 1));
     }
 }
 

@@ -53,22 +53,23 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaGetLastError();
 }
 
-template <int TR, int TC, bool ROW, bool COL>
+template <bool ROW, bool COL>
 static cudaError_t launch_msed_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed, DevView row,
                                        DevView col, float *P_row, float *P_col, uint32_t *amax_row,
                                        uint32_t *amax_col, cudaStream_t s) {
-    constexpr int kSmem = 2 * TR * TC * 2 + 1024;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(msed_kernel<TR, TC, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmem);
+        attr_err = cudaFuncSetAttribute(msed_kernel<ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        MsedCfg::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    const int64_t ntiles = (R / TR) * (C / TC);
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ntiles, sm_count()));
-    msed_kernel<TR, TC, ROW, COL><<<(unsigned)grid, 256, kSmem, s>>>(tmap, R, C, seed, row.codes, P_row, amax_row,
-                                                                    col.codes, P_col, amax_col);
+    const int64_t ntiles = (R >> 7) * (C >> 7);
+    // one CTA per SM; a single view needs two tiles per CTA to keep both halves busy
+    const int64_t per_cta = (ROW && COL) ? 1 : 2;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((ntiles + per_cta - 1) / per_cta, sm_count()));
+    msed_kernel<ROW, COL><<<(unsigned)grid, MsedCfg::kThreads, MsedCfg::kSmemBytes, s>>>(
+        tmap, R, C, seed, row.codes, P_row, amax_row, col.codes, P_col, amax_col);
     return cudaGetLastError();
 }
 
@@ -76,20 +77,10 @@ cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, boo
                               uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
                               uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s) {
     if (do_row && do_col)
-        return launch_msed_variant<128, 128, true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
-                                                         s);
-    if (do_row) {
-        if (R % 256 == 0)
-            return launch_msed_variant<256, 128, true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row,
-                                                              amax_col, s);
-        return launch_msed_variant<128, 128, true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row,
-                                                          amax_col, s);
-    }
-    if (C % 256 == 0)
-        return launch_msed_variant<128, 256, false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
-                                                          s);
-    return launch_msed_variant<128, 128, false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col,
-                                                      s);
+        return launch_msed_variant<true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+    if (do_row)
+        return launch_msed_variant<true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+    return launch_msed_variant<false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
 }
 
 cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
