@@ -60,9 +60,16 @@ __device__ __forceinline__ uint64_t shfl_xor1_u64(uint64_t v) {
     return r;
 }
 
-// Byte offset of tile element (r, c) in a 128x128 tile held as two 128x64 boxes (128-byte swizzle).
-__device__ __forceinline__ uint32_t tile_off(int r, int c) {
-    return (uint32_t)((c >> 6) * 16384 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+// Shared-memory loads at 32-bit shared addresses.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
 }
 
 // Butterfly strides 2..64 and quantization of one vector held by a thread pair.
@@ -247,14 +254,19 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         const int64_t tile = blockIdx.x + i * (int64_t)gridDim.x;
         const int64_t r0 = (tile / tiles_c) << 7, c0 = (tile % tiles_c) << 7;
         uint64_t P[32];
+        // A tile is two 128x64 boxes with the 128-byte swizzle: element (r, c) sits at byte
+        // (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
+        const uint32_t tbu = smem_u32(tb);
         if (rows) {
-            // row u, elements [64h, 64h + 64); register chunk c holds element chunk 8h + ((c + 4h) & 7)
+            // row u, elements [64h, 64h + 64); register chunk c holds element chunk 8h + (c ^ 4h),
+            // whose 16 bytes sit at swizzled chunk (c ^ 4h ^ (u % 8)) of row u in box h
+            const uint32_t rbase = tbu + h * 16384 + u * 128, rx = (uint32_t)((4 * h) ^ (u & 7)) << 4;
+            const uint32_t sbase = smem_u32(&sgn2[0]) + 256 * h, sx = 128 * h;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                const int e = 8 * h + ((c + 4 * h) & 7);
-                const uint4 v = *reinterpret_cast<const uint4 *>(tb + tile_off(u, 8 * e));
-                const uint4 m01 = *reinterpret_cast<const uint4 *>(&sgn2[4 * e]);
-                const uint4 m23 = *reinterpret_cast<const uint4 *>(&sgn2[4 * e + 2]);
+                const uint4 v = lds128(rbase + (rx ^ (uint32_t)(c << 4)));
+                const uint32_t sa = sbase + (sx ^ (uint32_t)(32 * c));
+                const uint4 m01 = lds128(sa), m23 = lds128(sa + 16);
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                 const uint32_t ml[4] = {m01.x, m01.z, m23.x, m23.z}, mh[4] = {m01.y, m01.w, m23.y, m23.w};
 #pragma unroll
@@ -265,19 +277,30 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
                 }
             }
         } else {
-            // column u, rows [64h, 64h + 64); slot j holds rows 2n, 2n + 1 of the half, n = (j + 16h) % 32
+            // column u, rows [64h, 64h + 64); slot j holds rows 2n, 2n + 1 of the half with
+            // n = (j + 16h) % 32, i.e. tile rows 96h + 2j (j < 16) and 32h + 2j (j >= 16).  The
+            // swizzle term depends on the row only through (2j + d) % 8, a constant per load.
+            const uint32_t colbase = (uint32_t)((u >> 6) * 16384 + (u & 7) * 2 + (((u & 63) >> 3) << 4));
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const int n = (j + 16 * h) & 31, rr = 64 * h + 2 * n;
-                const uint4 m = *reinterpret_cast<const uint4 *>(&sgn2[rr >> 1]);
-                const uint32_t u0 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr, u));
-                const uint32_t u1 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 1, u));
-                const uint32_t u2 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 2, u));
-                const uint32_t u3 = *reinterpret_cast<const uint16_t *>(tb + tile_off(rr + 3, u));
-                const float x0 = __uint_as_float((u0 << 16) + m.x), x1 = __uint_as_float((u1 << 16) + m.y);
-                const float x2 = __uint_as_float((u2 << 16) + m.z), x3 = __uint_as_float((u3 << 16) + m.w);
-                P[j] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
-                P[j + 1] = f2(__fadd_rn(x2, x3), __fsub_rn(x2, x3));
+            for (int half = 0; half < 2; ++half) {
+                const uint32_t hb = tbu + (half == 0 ? 12288u : 4096u) * h;
+                const uint32_t sb = smem_u32(&sgn2[0]) + (half == 0 ? 384u : 128u) * h;
+                uint32_t X[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) X[k] = hb + (colbase ^ (uint32_t)(k << 4));
+#pragma unroll
+                for (int jj = 0; jj < 16; jj += 2) {
+                    const int j = 16 * half + jj;
+                    const uint4 m = lds128(sb + 8 * j);
+                    const uint32_t u0 = lds16(X[(2 * j) & 7] + 256 * j);
+                    const uint32_t u1 = lds16(X[(2 * j + 1) & 7] + 256 * j + 128);
+                    const uint32_t u2 = lds16(X[(2 * j + 2) & 7] + 256 * j + 256);
+                    const uint32_t u3 = lds16(X[(2 * j + 3) & 7] + 256 * j + 384);
+                    const float x0 = __uint_as_float((u0 << 16) + m.x), x1 = __uint_as_float((u1 << 16) + m.y);
+                    const float x2 = __uint_as_float((u2 << 16) + m.z), x3 = __uint_as_float((u3 << 16) + m.w);
+                    P[j] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
+                    P[j + 1] = f2(__fadd_rn(x2, x3), __fsub_rn(x2, x3));
+                }
             }
         }
         // The tile is in registers: release the stage; the last warp to do so refills it.
