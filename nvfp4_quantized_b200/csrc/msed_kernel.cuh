@@ -50,6 +50,30 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return r;
 }
 
+// a / 6 rounded to nearest-even, for normal a >= 2^-100: q0 = a * RN(1/6), the remainder
+// a - 6 q0 is exact in one FMA, and one FMA correction q0 + rem * RN(1/6) rounds to RN(a/6)
+// (Markstein's correction step; verified exhaustively over every significand of a binade and
+// over the extreme binades of the range, and exact scaling by powers of two extends it to all
+// a in [2^-100, 2^128)).
+__device__ __forceinline__ float div6_rn(float a) {
+    constexpr float kSixth = 0.16666667163372039794921875f;   // RN(1/6) = 0x3E2AAAAB
+    const float q0 = __fmul_rn(a, kSixth);
+    const float rem = __fmaf_rn(-q0, 6.0f, a);
+    return __fmaf_rn(rem, kSixth, q0);
+}
+
+// max(|a|, |b|, |c|) (sm_100a three-input max; exact, so the grouping does not matter)
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint64_t shfl_xor1_u64(uint64_t v) {
     uint32_t lo, hi;
     asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
@@ -115,18 +139,14 @@ __device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint
         float y[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) f2_split(P[8 * g + i], y[2 * i], y[2 * i + 1]);
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1]));
-#pragma unroll
-        for (int w = 8; w > 1; w >>= 1) {
-#pragma unroll
-            for (int i = 0; i < w / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
-        }
-        const float a = m8[0];     // max is exact: the evaluation order does not matter
+        // max is exact: the evaluation order does not matter
+        const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
+        const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
+        const float m4 = absmax3(y[12], y[13], y[14]);
+        const float a = fmaxf(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
         amax = fmaxf(amax, a);
         const bool live = a >= kTiny;
-        const float p = live ? __fdiv_rn(a, 6.0f) : 0.0f;
+        const float p = live ? div6_rn(a) : 0.0f;
         const float r = live ? __frcp_rn(p) : 0.0f;          // flushed group: sign-preserving zeros
         const uint64_t rr = f2(r, r);
         float v[16];
