@@ -5,38 +5,53 @@
 // C = alpha * gA * gB * sum_k val(A) sA * val(B) sB, both operands K-major, fp32 accumulation.
 //
 // Why a pair: with one SM per 128x256 tile, every SM streams 216 KB of operands per K = 256
-// step from L2, and the mainloop is bound by that stream (about 7.4 TB/s of TMA traffic on
-// B200), not by the tensor cores.  A CTA pair computes a 256x256 tile with one
-// tcgen05.mma.cta_group::2: each SM holds its own 128 rows of A and one half (128 rows) of B,
-// so each SM streams 1.5x fewer bytes per flop.  Operand loads are plain TMA loads (no
-// multicast) whose completion both SMs report to the leader SM's barrier.
+// step from L2.  A CTA pair computes a 256x256 tile with one tcgen05.mma.cta_group::2: each SM
+// holds its own 128 rows of A and one half (128 rows) of B, so each SM streams 1.5x fewer bytes
+// per flop.  Operand loads are plain TMA loads (no multicast) whose completion both SMs report to
+// the leader SM's barrier.
 //
-// Roles, per CTA of 320 threads (10 warps), persistent over 256x256 tiles:
-//   warp 0, one thread : producer.  Waits for a free stage (its own "empty" barrier); the
-//                        leader arms the stage's "full" barrier with both SMs' code bytes; both
-//                        load A (own 128 rows) and B (own 128 of the 256 rows) reporting to the
-//                        leader, and their scale atoms (A: own rows; B: all 256 rows, because
-//                        each SM's tensor memory needs the scales of every B column) reporting
-//                        to their own "sf_full" barrier.
+// What bounds the pipeline on B200 (measured with timing-only variants of this kernel, dgrad
+// shape 16384 x 2048 x 8192): the MMA stream alone runs at ~7 PFLOP/s; the code loads alone
+// (5-stage ring, released by tcgen05.commit) stream ~12 TB/s into the SMs, because a TMA load
+// takes ~2 us under full load and the ring keeps ~190 KB in flight per SM.  What is left is the
+// scale path: the 12 tcgen05.cp of a stage cost ~33 ns each when the MMA thread issues them,
+// overlap the MMAs when another thread does, but then sit on the critical path between a
+// stage's MMAs retiring (its TMEM scale region) and the next use of that region; handing the
+// scales over through tcgen05.st from registers is slower still.  The best arrangement found:
+// the scales travel in their own deeper ring, two stages ahead of the codes, and a copier
+// thread moves them as soon as a region frees (~2.9 PFLOP/s on that shape, ~50% of a library
+// NVFP4 GEMM on the same GPU).
+//
+// Roles, per CTA of 384 threads (12 warps), persistent over 256x256 tiles (K = 256 per stage):
+//   warp 0, lanes 0..9 : code producers, one thread per operand and ring slot (TMA loads issued
+//                        by one thread are processed one after another).  Lane s loads A, lane
+//                        5 + s loads B of code slot s: own 128 rows of A and own 128 of the 256
+//                        B rows, reported to the leader's "full" barrier after the slot's
+//                        "empty" (the MMAs that read it) completed.
+//   warp 3, lanes 0..6 : scale producers (a warp of their own: lanes of one warp that wait on
+//                        different barriers slow each other down).  Lane q loads SFA and SFB of
+//                        scale slot q (A: own rows; B: all 256 rows, because each SM's tensor
+//                        memory needs the scales of every B column) into the leader's "sf_full"
+//                        after "sf_free" (the copies that read it) completed.
 //   warp 1             : allocates/frees 512 TMEM columns (both SMs); on the leader, one thread
-//                        issues the four 256x256x64 MMAs of each stage and a tcgen05.commit that
-//                        frees the stage on both SMs.  Nothing else sits in the MMA pipe.
-//   warps 2..5         : scale writers.  Warp w owns TMEM lane quadrant w%4: it reads the
-//                        stage's scale atoms from shared memory and stores them with tcgen05.st
-//                        into that stage's scale region of tensor memory, in the replicated
-//                        layout the block-scaled MMA reads, then reports to the leader.
-//                        (Moving them with tcgen05.cp instead costs the MMA pipe ~65 cycles per
-//                        copy, 12 copies per stage -- more than the MMAs themselves.)
-//   warps 6..9         : epilogue.  Warp w reads TMEM lane quadrant w%4 (all 256 columns) in
-//                        32-column chunks and scales them.  bf16 output goes to a per-warp
-//                        staging region of shared memory; the accumulator is released and TMA
-//                        stores write the block out while the next tile's MMAs run.  fp32
-//                        output (1 KB per row) is stored chunk by chunk, released after the
-//                        last read.
-// Tensor memory: accumulator columns [0, 256); scale region of stage s at 256 + 48 s
-// (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
-// Every wait is bounded; on a timeout the CTA records QT2_ERR_TIMEOUT, both CTAs drain the
-// loads they issued that were not consumed, meet at the final cluster barrier and free TMEM.
+//                        issues the four 256x256x64 MMAs of each stage after "full" and "sftm"
+//                        and a tcgen05.commit that frees the code slot (and the stage's scale
+//                        region of TMEM) on both SMs.
+//   warp 2, leader     : scale copier.  For stage j: waits "sf_full" of scale slot j % 7 and the
+//                        MMAs of stage j - 5 (its TMEM scale region), copies the 12 scale atoms
+//                        from both SMs' shared memory into their tensor memory (tcgen05.cp
+//                        32x128b, replicated into the four lane quadrants, the layout the
+//                        block-scaled MMA reads), then commits to "sftm" of region j % 5 and to
+//                        "sf_free" of the scale slot on both SMs.
+//   warps 4..11        : epilogue.  Warp w reads TMEM lane quadrant w%4, columns [0, 128) for
+//                        warps 4..7 and [128, 256) for warps 8..11, in 32-column chunks, scales
+//                        them and stores its rows straight to global memory (bf16 or fp32); the
+//                        accumulator is released right after its last tensor-memory read.
+// Tensor memory: accumulator columns [0, 256); scale region r (of stage j, r = j % 5) at
+// 256 + 48 r (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
+// Every wait is bounded; on a timeout the CTA records QT2_ERR_TIMEOUT, the leader drains the
+// loads and tensor-core work that were issued, both CTAs meet at the final cluster barrier and
+// free TMEM.
 #pragma once
 
 #include "qt2_device.cuh"
@@ -123,38 +138,57 @@ __device__ __forceinline__ void tc_mma_pair_nvfp4(uint32_t d_tmem, uint64_t ades
         : "memory");
 }
 
+// Copy one 512-byte scale atom (32 rows x 16 bytes) from shared memory into 32 TMEM lanes x 4
+// columns, replicated into all four lane quadrants, in both CTAs of the pair (each from its own
+// shared memory at the same address).
+__device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Arrive on `bar` of the leader CTA only once this thread's tcgen05 work so far has completed.
+__device__ __forceinline__ void tc_commit_pair_leader(uint32_t bar) {
+    const uint16_t leader_only = 0x1;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                     bar),
+                 "h"(leader_only)
+                 : "memory");
+}
+
 // ------------------------------------------------------------------ configuration
 struct Gemm2Cfg {
-    static constexpr int kStages = 4;
-    static constexpr int kThreads = 320;
-    static constexpr int kSfWarps = 4;
-    static constexpr int kEpiWarps = 4;
+    static constexpr int kStages = 5;             // code ring (A + B)
+    static constexpr int kSfStages = 7;           // scale ring, loaded up to 2 stages ahead
+    static constexpr int kThreads = 384;
+    static constexpr int kEpiWarp0 = 4;
+    static constexpr int kEpiWarps = 8;
     static constexpr int kA = 128 * 128;          // own 128 rows x 128 bytes (K = 256)
     static constexpr int kB = 128 * 128;          // own half of the 256 B rows
     static constexpr int kSfa = 4 * 512;          // 4 k-blocks x one 512-byte atom
     static constexpr int kSfb = 2 * 4 * 512;      // both 128-row atoms of B, 4 k-blocks each
-    static constexpr int kStageBytes = kA + kB + kSfa + kSfb;   // 38912 = 38 KB, keeps 1 KB alignment
-    static constexpr int kStagingBytes = 4 * 32 * 512;   // bf16 output: 4 epilogue warps x 32 rows x 256 cols
-    static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 256;
-    static constexpr int kTmemCols = 512;         // accumulator 256 + 4 stage scale regions x 48
+    static constexpr int kStageBytes = kA + kB;   // 32 KB, keeps 1 KB alignment
+    static constexpr int kSfStageBytes = kSfa + kSfb;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kSfStages * kSfStageBytes + 1024 + 512;
+    static constexpr int kTmemCols = 512;         // accumulator 256 + 5 scale regions x 48
     static constexpr int kSfRegionCols = 48;
     // E2M1 x E2M1, UE4M3 scales, K-major A and B, M = 256 (pair), N = 256
     static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (32u << 17) | (16u << 24);
 };
+static_assert(Gemm2Cfg::kStages * 2 <= 32 && Gemm2Cfg::kSfStages <= 32, "producer lanes");
+static_assert(256 + Gemm2Cfg::kStages * Gemm2Cfg::kSfRegionCols <= Gemm2Cfg::kTmemCols, "TMEM columns");
+
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                           const __grid_constant__ CUtensorMap tmC, const float *__restrict__ gA, const float *__restrict__ gB, float alpha,
+                           const float *__restrict__ gA, const float *__restrict__ gB, float alpha,
                            void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype) {
     using Cfg = Gemm2Cfg;
-    constexpr int S = Cfg::kStages;
+    constexpr int S = Cfg::kStages, SF = Cfg::kSfStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint8_t *staging = base + S * Cfg::kStageBytes;   // bf16 output tile, one 16 KB region per epilogue warp
-    // barriers: full[S] sf_full[S] sf_ready[S] empty[S] acc_full acc_empty
-    uint64_t *bars = reinterpret_cast<uint64_t *>(staging + Cfg::kStagingBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 2);
+    uint8_t *sf_base = base + S * Cfg::kStageBytes;
+    // barriers: full[S] sftm[S] empty[S] sf_full[SF] sf_free[SF] acc_full acc_empty
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sf_base + SF * Cfg::kSfStageBytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 2 * SF + 2);
     int *consumed_slot = reinterpret_cast<int *>(tmem_slot + 1);
 
     const uint32_t rank = cluster_ctarank();
@@ -163,17 +197,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     const int num_pn = N >> 8, tiles = (M >> 8) * num_pn;
     const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
     const int nkb = K >> 6, nks = (nkb + 3) >> 2;
-    const uint32_t full0 = smem_u32(bars), sf_full0 = smem_u32(bars + S), sf_ready0 = smem_u32(bars + 2 * S),
-                   empty0 = smem_u32(bars + 3 * S);
-    const uint32_t acc_full = smem_u32(bars + 4 * S), acc_empty = smem_u32(bars + 4 * S + 1);
+    const int my_tiles = tiles > cluster_id ? (tiles - 1 - cluster_id) / num_clusters + 1 : 0;
+    const int total = my_tiles * nks;   // stages this pair runs
+    const uint32_t full0 = smem_u32(bars), sftm0 = smem_u32(bars + S), empty0 = smem_u32(bars + 2 * S);
+    const uint32_t sf_full0 = smem_u32(bars + 3 * S), sf_free0 = smem_u32(bars + 3 * S + SF);
+    const uint32_t acc_full = smem_u32(bars + 3 * S + 2 * SF), acc_empty = acc_full + 8;
 
     if (threadIdx.x == 0) {
         *consumed_slot = 0;
         for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(sf_full0 + 8 * s, 1);
-            mbar_init(sf_ready0 + 8 * s, 2 * Cfg::kSfWarps);
-            mbar_init(empty0 + 8 * s, 1);
+            mbar_init(full0 + 8 * s, 2);    // the A and B issuers of the leader
+            mbar_init(sftm0 + 8 * s, 1);    // the scale copier's commit
+            mbar_init(empty0 + 8 * s, 1);   // the MMA thread's commit
+        }
+        for (int q = 0; q < SF; ++q) {
+            mbar_init(sf_full0 + 8 * q, 1);   // the scale issuer of the leader
+            mbar_init(sf_free0 + 8 * q, 1);   // the scale copier's commit
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * Cfg::kEpiWarps);
@@ -188,52 +227,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int issued = 0;
-    if (warp == 0 && lane == 0) {
-        // -------------------------------------------------------------- producer (both CTAs)
-        prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
-        prefetch_tmap(&tmSFA);
-        prefetch_tmap(&tmSFB);
+    auto stage_tile = [&](int it, int &pm, int &pn, int &ks) {
+        const int tile = cluster_id + (it / nks) * num_clusters;
+        ks = it % nks;
+        pm = tile / num_pn;
+        pn = tile - pm * num_pn;
+    };
+
+    int issued = 0, sf_issued = 0;   // producers: code / scale stages whose loads this lane issued
+    int mma_done = 0;                // MMA thread: stages whose MMAs were issued
+    int copied = 0;                  // copier: stages whose scales were copied
+    if (warp == 0 && lane < 2 * S) {
+        // -------------------------------------------------------------- code producers (both CTAs)
+        const int op = lane / S, slot = lane % S;
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            prefetch_tmap(&tmB);
+        }
         const uint32_t full_leader0 = mapa_shared(full0, 0);
-        bool ok = true;
-        int it = 0;
-        for (int tile = cluster_id; tile < tiles && ok; tile += num_clusters) {
-            const int pm = tile / num_pn, pn = tile - pm * num_pn;
-            const int32_t a_row = pm * 256 + (int)rank * 128, b_row = pn * 256 + (int)rank * 128;
-            const int32_t sfa_row = pm * 2 + (int)rank, sfb_row = pn * 2;
-            for (int ks = 0; ks < nks; ++ks, ++it) {
-                const int s = it % S;
-                if (it >= S && !mbar_wait(empty0 + 8 * s, ((it / S) & 1) ^ 1)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t fb = full_leader0 + 8 * s, sfb_bar = sf_full0 + 8 * s;
-                if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * (Cfg::kA + Cfg::kB));
-                mbar_arrive_expect_tx(sfb_bar, Cfg::kSfa + Cfg::kSfb);
-                uint8_t *st = base + s * Cfg::kStageBytes;
-                tma_load_2d_pair(smem_u32(st), &tmA, ks * 128, a_row, fb);
-                tma_load_2d_pair(smem_u32(st + Cfg::kA), &tmB, ks * 128, b_row, fb);
-                tma_load_2d(smem_u32(st + Cfg::kA + Cfg::kB), &tmSFA, ks * 256, sfa_row, sfb_bar);
-                tma_load_2d(smem_u32(st + Cfg::kA + Cfg::kB + Cfg::kSfa), &tmSFB, ks * 256, sfb_row, sfb_bar);
-                issued = it + 1;
-            }
+        for (int it = slot; it < total; it += S) {
+            if (it >= S && !mbar_wait(empty0 + 8 * slot, ((it / S) & 1) ^ 1)) break;
+            int pm, pn, ks;
+            stage_tile(it, pm, pn, ks);
+            const uint32_t dst = smem_u32(base + slot * Cfg::kStageBytes + (op ? Cfg::kA : 0));
+            if (leader) mbar_arrive_expect_tx(full0 + 8 * slot, 2 * (op ? Cfg::kB : Cfg::kA));
+            if (op == 0)
+                tma_load_2d_pair(dst, &tmA, ks * 128, pm * 256 + (int)rank * 128, full_leader0 + 8 * slot);
+            else
+                tma_load_2d_pair(dst, &tmB, ks * 128, pn * 256 + (int)rank * 128, full_leader0 + 8 * slot);
+            issued = it + 1;
+        }
+    } else if (warp == 3 && lane < SF) {
+        // -------------------------------------------------------------- scale producers (both CTAs)
+        const int q = lane;
+        if (q == 0) {
+            prefetch_tmap(&tmSFA);
+            prefetch_tmap(&tmSFB);
+        }
+        const uint32_t sf_full_leader0 = mapa_shared(sf_full0, 0);
+        for (int j = q; j < total; j += SF) {
+            if (j >= SF && !mbar_wait(sf_free0 + 8 * q, ((j / SF) & 1) ^ 1)) break;
+            int pm, pn, ks;
+            stage_tile(j, pm, pn, ks);
+            const uint32_t dst = smem_u32(sf_base + q * Cfg::kSfStageBytes);
+            if (leader) mbar_arrive_expect_tx(sf_full0 + 8 * q, 2 * (Cfg::kSfa + Cfg::kSfb));
+            tma_load_2d_pair(dst, &tmSFA, ks * 256, pm * 2 + (int)rank, sf_full_leader0 + 8 * q);
+            tma_load_2d_pair(dst + Cfg::kSfa, &tmSFB, ks * 256, pn * 2, sf_full_leader0 + 8 * q);
+            sf_issued = j + 1;
         }
     } else if (warp == 1 && lane == 0 && leader) {
         // -------------------------------------------------------------- MMA issuer (leader)
+        int it = 0;
         bool ok = true;
-        int it = 0, t_iter = 0;
-        for (int tile = cluster_id; tile < tiles && ok; tile += num_clusters, ++t_iter) {
+        for (int t_iter = 0; t_iter < my_tiles && ok; ++t_iter) {
             if (t_iter > 0 && !mbar_wait(acc_empty, (t_iter - 1) & 1)) break;
             tc_fence_after();
             for (int ks = 0; ks < nks; ++ks, ++it) {
                 const int s = it % S;
                 const uint32_t par = (it / S) & 1;
-                if (!mbar_wait(full0 + 8 * s, par) || !mbar_wait(sf_ready0 + 8 * s, par)) {
+                if (!mbar_wait(full0 + 8 * s, par) || !mbar_wait(sftm0 + 8 * s, par)) {
                     ok = false;
                     break;
                 }
-                *consumed_slot = it + 1;
                 tc_fence_after();
                 const int nk = min(4, nkb - ks * 4);
                 const uint32_t st = smem_u32(base + s * Cfg::kStageBytes);
@@ -245,107 +300,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                                       (ks | kk) != 0);
                 }
                 tc_commit_pair_both(empty0 + 8 * s);
+                mma_done = it + 1;
+                *consumed_slot = it + 1;
             }
-            tc_commit_pair_both(acc_full);
+            if (ok) tc_commit_pair_both(acc_full);
         }
-    } else if (warp >= 2 && warp < 2 + Cfg::kSfWarps) {
-        // -------------------------------------------------------------- scale writers (both CTAs)
-        // Lane r of the warp owning quadrant q writes TMEM lane 32q + r.  In the replicated layout
-        // the MMA reads, that lane's 4 columns of an A k-block hold atom row r (rows r, r+32, r+64,
-        // r+96 of the 128-row block, 4 scales each); its 8 columns of a B k-block hold row r of the
-        // two B atoms (B rows n and n+128 of the 256-column tile).
-        const int quad = warp & 3;
-        const uint32_t sf_ready_leader0 = mapa_shared(sf_ready0, 0);
-        int it = 0;
-        bool ok = true;
-        for (int tile = cluster_id; tile < tiles && ok; tile += num_clusters) {
-            for (int ks = 0; ks < nks; ++ks, ++it) {
-                const int s = it % S;
-                if (!mbar_wait(sf_full0 + 8 * s, (it / S) & 1)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t *sfa_s = base + s * Cfg::kStageBytes + Cfg::kA + Cfg::kB;
-                const uint8_t *sfb_s = sfa_s + Cfg::kSfa;
-                // va: A k-blocks 0..3 (4 words each); vb[j]: B k-blocks 2j and 2j+1 (8 words each:
-                // 4 from the first B atom, 4 from the second)
-                uint32_t va[16], vb[2][16];
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const uint4 a = *reinterpret_cast<const uint4 *>(sfa_s + kb * 512 + lane * 16);
-                    va[4 * kb + 0] = a.x;
-                    va[4 * kb + 1] = a.y;
-                    va[4 * kb + 2] = a.z;
-                    va[4 * kb + 3] = a.w;
-                    const uint4 b0 = *reinterpret_cast<const uint4 *>(sfb_s + kb * 512 + lane * 16);
-                    const uint4 b1 = *reinterpret_cast<const uint4 *>(sfb_s + 2048 + kb * 512 + lane * 16);
-                    const int j = kb >> 1, o = 8 * (kb & 1);
-                    vb[j][o + 0] = b0.x;
-                    vb[j][o + 1] = b0.y;
-                    vb[j][o + 2] = b0.z;
-                    vb[j][o + 3] = b0.w;
-                    vb[j][o + 4] = b1.x;
-                    vb[j][o + 5] = b1.y;
-                    vb[j][o + 6] = b1.z;
-                    vb[j][o + 7] = b1.w;
-                }
-                const uint32_t t_sf = tmem + ((uint32_t)(quad * 32) << 16) + 256 + Cfg::kSfRegionCols * s;
-                tmem_st_32x32b_x16(t_sf, va);
-                tmem_st_32x32b_x16(t_sf + 16, vb[0]);
-                tmem_st_32x32b_x16(t_sf + 32, vb[1]);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(sf_ready_leader0 + 8 * s);
+    } else if (warp == 2 && lane == 0 && leader) {
+        // -------------------------------------------------------------- scale copier (leader)
+        // A k-block's A scales are one atom (TMEM columns +4kb), its B scales two atoms (the B
+        // rows n and n + 128 of the tile; columns +16+8kb and +20+8kb).
+        for (int j = 0; j < total; ++j) {
+            const int q = j % SF, r = j % S;
+            if (!mbar_wait(sf_full0 + 8 * q, (j / SF) & 1)) break;
+            if (j >= S && !mbar_wait(empty0 + 8 * r, ((j / S) & 1) ^ 1)) break;   // region r is free
+            tc_fence_after();
+            const int nk = min(4, nkb - (j % nks) * 4);
+            const uint32_t sfa = smem_u32(sf_base + q * Cfg::kSfStageBytes);
+            const uint32_t sfb = sfa + Cfg::kSfa;
+            const uint32_t t_sf = tmem + 256 + Cfg::kSfRegionCols * r;
+            for (int kk = 0; kk < nk; ++kk) {
+                tc_cp_pair_32x128b_warpx4(t_sf + 4 * kk, make_smem_desc(sfa + 512 * kk, 0, 128, 0));
+                tc_cp_pair_32x128b_warpx4(t_sf + 16 + 8 * kk, make_smem_desc(sfb + 512 * kk, 0, 128, 0));
+                tc_cp_pair_32x128b_warpx4(t_sf + 20 + 8 * kk, make_smem_desc(sfb + 2048 + 512 * kk, 0, 128, 0));
             }
+            tc_commit_pair_leader(sftm0 + 8 * r);
+            tc_commit_pair_both(sf_free0 + 8 * q);
+            copied = j + 1;
         }
-    } else if (warp >= 2 + Cfg::kSfWarps) {
+    } else if (warp >= Cfg::kEpiWarp0) {
         // -------------------------------------------------------------- epilogue (both CTAs)
-        const int quad = warp & 3;
+        const int quad = warp & 3, ew = warp - Cfg::kEpiWarp0;
+        const int cb = (ew >> 2) * 128;   // this warp's 128 of the tile's 256 columns
         const uint32_t acc_empty_leader = mapa_shared(acc_empty, 0);
         const float sc = alpha * (*gA) * (*gB);
-        int t_iter = 0;
-        for (int tile = cluster_id; tile < tiles; tile += num_clusters, ++t_iter) {
-            if (!mbar_wait(acc_full, t_iter & 1)) break;
+        for (int t_iter = 0; t_iter < my_tiles; ++t_iter) {
+            if (!mbar_wait_warp(acc_full, t_iter & 1)) break;
             tc_fence_after();
+            const int tile = cluster_id + t_iter * num_clusters;
             const int pm = tile / num_pn, pn = tile - pm * num_pn;
             const int64_t row = (int64_t)pm * 256 + rank * 128 + quad * 32 + lane;
-            const int64_t col = (int64_t)pn * 256;
-            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
-            if (c_dtype == QT2_DTYPE_F32) {
-                // fp32 row (1 KB): 32-column chunks stored as they are read; the accumulator is
-                // released right after the last tensor-memory read
+            const int64_t col = (int64_t)pn * 256 + cb;
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + cb;
 #pragma unroll 1
-                for (int c = 0; c < 256; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld_32x32b_x16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_ld_wait();
-                    if (c == 224) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
-                    }
+            for (int c = 0; c < 128; c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                tmem_ld_32x32b_x16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+                tmem_ld_wait();
+                if (c == 96) {   // last read of this tile: release the accumulator
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+                }
+                if (c_dtype == QT2_DTYPE_F32) {
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + row * ldc + col + c);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         dst[i] = make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
                                              __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc);
-                }
-            } else {
-                // bf16: the warp's 32 x 256 block goes to its staging region as four 32-row x 64-column
-                // boxes (128-byte swizzle), the accumulator is released, then TMA stores write it out
-                uint8_t *stg = staging + (warp - 2 - Cfg::kSfWarps) * 16384;
-                if (t_iter > 0) {
-                    if (lane == 0) bulk_wait_read_all();   // the previous tile's stores have read it
-                    __syncwarp();
-                }
-#pragma unroll 1
-                for (int c = 0; c < 256; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld_32x32b_x16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_ld_wait();
+                } else {
                     uint32_t p[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -353,38 +366,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                                                                   __uint_as_float(v[2 * i + 1]) * sc);
                         p[i] = *reinterpret_cast<uint32_t *>(&b2);
                     }
-                    uint8_t *box = stg + (c >> 6) * 4096 + lane * 128;
-                    const int k0 = (c & 63) >> 3;
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(Cout) + row * ldc + col + c);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        *reinterpret_cast<uint4 *>(box + (((k0 + i) ^ (lane & 7)) << 4)) =
-                            make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                }
-                tc_fence_before();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_remote(acc_empty_leader);
-                    const int32_t y0 = (int32_t)(row - lane);
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) tma_store_2d(&tmC, smem_u32(stg + b * 4096), (int32_t)col + 64 * b, y0);
-                    bulk_commit();
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
                 }
             }
         }
-        if (lane == 0) bulk_wait_all();   // this warp's output stores are complete
     }
+    issued = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)issued);
+    sf_issued = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)sf_issued);
     __syncwarp();
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();   // both CTAs are done; the leader's consumed count is final
-    if (warp == 0 && lane == 0) {
-        // Only after a timeout can issued loads still be in flight: wait (bounded) for them.
-        const int consumed = (int)ld_shared_cluster_u32(mapa_shared(smem_u32(consumed_slot), 0));
-        for (int it = consumed; it < issued; ++it) {
-            if (leader) mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
-            mbar_wait(sf_full0 + 8 * (it % S), (it / S) & 1);
-        }
+    cluster_sync_all();   // both CTAs are done issuing; the leader's counts are final
+    if (leader && threadIdx.x == 0) {
+        // Only after a timeout can work still be in flight: wait (bounded) for every issued
+        // stage's code loads ...
+        for (int it = *consumed_slot; it < issued; ++it) mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
+    }
+    if (leader && warp == 3 && lane == 0) {
+        // ... and scale loads (the newest one of each slot; older ones were copied)
+        for (int j = sf_issued > SF ? sf_issued - SF : 0; j < sf_issued; ++j)
+            mbar_wait(sf_full0 + 8 * (j % SF), (j / SF) & 1);
+    }
+    if (leader && warp == 2 && lane == 0 && copied > 0) {
+        const int j = copied - 1;
+        mbar_wait(sf_free0 + 8 * (j % SF), (j / SF) & 1);
+    }
+    if (leader && warp == 1 && lane == 0 && mma_done > 0) {
+        const int it = mma_done - 1;
+        mbar_wait(empty0 + 8 * (it % S), (it / S) & 1);
     }
     cluster_sync_all();   // no SM frees TMEM or exits while its pair may still touch it
     tc_fence_after();

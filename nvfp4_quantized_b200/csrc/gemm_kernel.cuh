@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
 
     // -------------------------------------------------------------------- epilogue
-    const bool acc_ok = mbar_wait(accum_bar, 0);
+    const bool acc_ok = mbar_wait_warp(accum_bar, 0);
     tc_fence_after();
     if (acc_ok) {
         const float sc = alpha * (*gA) * (*gB);

@@ -179,6 +179,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
+// Bounded wait by a whole warp, for warps that go on to warp-collective (.sync.aligned)
+// tcgen05 instructions: every lane polls, and the vote reconverges the warp and makes the
+// outcome uniform (false if any lane gave up).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity));
+}
+
 // 2D tiled TMA load (no multicast) of box {x, y} into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t x, int32_t y, uint32_t bar) {
     asm volatile(

@@ -38,7 +38,7 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, De
                               int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s);
 
 cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
-                                   const CUtensorMap &tmSFB, const CUtensorMap &tmC, DevView a, DevView b, int64_t M,
+                                   const CUtensorMap &tmSFB, DevView a, DevView b, int64_t M,
                                    int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
                                    cudaStream_t s);
 

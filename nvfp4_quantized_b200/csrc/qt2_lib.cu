@@ -117,7 +117,7 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, De
 }
 
 cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
-                                   const CUtensorMap &tmSFB, const CUtensorMap &tmC, DevView a, DevView b, int64_t M,
+                                   const CUtensorMap &tmSFB, DevView a, DevView b, int64_t M,
                                    int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
                                    cudaStream_t s) {
     static std::once_flag once;
@@ -130,7 +130,7 @@ cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tm
     const int64_t tiles = (M / 256) * (N / 256);
     const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count() / 2));
     gemm_nvfp4_pair_kernel<<<(unsigned)(2 * clusters), Gemm2Cfg::kThreads, Gemm2Cfg::kSmemBytes, s>>>(
-        tmA, tmB, tmSFA, tmSFB, tmC, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype);
+        tmA, tmB, tmSFA, tmSFB, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype);
     return cudaGetLastError();
 }
 
@@ -285,7 +285,7 @@ qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, f
     CUtensorMap tmA, tmB;
     if (M % 256 == 0 && N % 256 == 0) {
         // pair kernel: 128-row code boxes per SM, scale atoms as rows of K/64 512-byte atoms
-        CUtensorMap tmSFA, tmSFB, tmC;
+        CUtensorMap tmSFA, tmSFB;
         if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
                             128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b.codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
@@ -295,15 +295,7 @@ qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, f
             !encode_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT64, b.scales, (uint64_t)K, (uint64_t)N / 128,
                             (uint64_t)K * 8, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
             return QT2_ERR_CUDA;
-        // bf16 output leaves through TMA stores of 32-row x 64-column boxes (unused for fp32 output)
-        if (c_dtype == QT2_DTYPE_BF16) {
-            if (!encode_tmap_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c, (uint64_t)N, (uint64_t)M, (uint64_t)ldc * 2,
-                                64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
-                return QT2_ERR_CUDA;
-        } else {
-            std::memset(&tmC, 0, sizeof(tmC));
-        }
-        return from_cuda(launch_gemm_nvfp4_pair(tmA, tmB, tmSFA, tmSFB, tmC, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
+        return from_cuda(launch_gemm_nvfp4_pair(tmA, tmB, tmSFA, tmSFB, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
     }
     const int bn = (N % 256 == 0) ? 256 : 128;
     if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
