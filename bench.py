@@ -55,39 +55,62 @@ def peaks():
 
 # ---------------------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples the SM clock, power and clock-event reasons through NVML every few ms while the
-    timed region runs (read-only queries; no setting is touched)."""
+    """Samples the SM clock, power and clock-event reasons through NVML every 2 ms while the
+    timed region runs (read-only queries; no setting is touched).  NVML is opened and the
+    sampling thread started before the warm-up, so the whole timed region is covered; the
+    region's first and last samples are taken synchronously by begin() and end()."""
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index: int, period_s: float = 0.005):
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
+        import threading
         self.gpu, self.period = gpu_index, period_s
         self.samples = []
-        self._stop = None
+        self.max_mhz, self.error, self._h = None, None, None
+        self._ready, self._stop, self._rec = threading.Event(), threading.Event(), threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        import pynvml
+        sm = pynvml.nvmlDeviceGetClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        pw = pynvml.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        self.samples.append((sm, pw, rs))
 
     def _run(self):
-        import pynvml
         try:
+            import pynvml
             pynvml.nvmlInit()
-            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-            while not self._stop.is_set():
-                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
-                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((sm, pw, rs))
-                self._stop.wait(self.period)
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception as e:   # NVML unavailable: report that, never fail the run
             self.error = repr(e)
+            self._ready.set()
+            return
+        self._ready.set()
+        while not self._stop.is_set():
+            if self._rec.is_set():
+                try:
+                    self._sample()
+                except Exception as e:
+                    self.error = repr(e)
+            self._stop.wait(self.period)
 
-    def __enter__(self):
-        import threading
-        self.max_mhz, self.error = None, None
-        self._stop = threading.Event()
-        self._t = threading.Thread(target=self._run, daemon=True)
+    def start(self):
         self._t.start()
         return self
 
-    def __exit__(self, *a):
+    def begin(self):
+        self._ready.wait(timeout=30)
+        if self._h is not None:
+            self._sample()
+        self._rec.set()
+
+    def end(self):
+        self._rec.clear()
+        if self._h is not None:
+            self._sample()
+
+    def stop(self):
         self._stop.set()
         self._t.join(timeout=5)
 
@@ -100,7 +123,7 @@ class ClockSampler:
         reasons = sorted({n for s in loaded for n, bit in self.REASONS.items() if s[2] & bit})
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
                 "samples": len(self.samples), "samples_under_load": len(loaded),
-                "power_w_max": max(s[1] for s in self.samples), "source": "nvml, 5 ms period"}
+                "power_w_max": max(s[1] for s in self.samples), "source": "nvml, 2 ms period"}
 
 
 # ---------------------------------------------------------------------------------------- our arm
@@ -166,6 +189,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
 
+    clk = ClockSampler(local_rank).start()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -174,14 +198,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i, events[i])
-        t_end.record(stream)
-        torch.cuda.synchronize()
+    clk.begin()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk.end()
+    clk.stop()
     barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     status = Q.qt2_device_status(stream)
@@ -326,7 +352,7 @@ def main():
             with open(prof) as f:
                 tj = json.load(f)
             import hashlib
-            src = os.path.join(ROOT, "nvfp4_quantized_b200", "csrc", "gemm_kernel.cuh")
+            src = os.path.join(ROOT, "nvfp4_quantized_b200", "csrc", "gemm2_kernel.cuh")
             sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
             if tj.get("config") == args.config and tj.get("kernel_sha1") == sha:
                 traffic = tj.get("bytes_per_launch")   # counters of the current kernel only
@@ -364,7 +390,7 @@ def main():
                    "output": "Y bf16, dX bf16, dW fp32"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp4_peak, "traffic": traffic,
-                     "kernel": "gemm_nvfp4 (mean of the fwd, dgrad and wgrad launches)",
+                     "kernel": "gemm_nvfp4_pair_kernel (mean of the fwd, dgrad and wgrad launches)",
                      "peak_source": f"{pk['source']}: sustained bf16 {pk['bf16_sustained']} TFLOP/s x 4 "
                                     "(nominal dense fp4/bf16 ratio)"},
         "quantizers": {"gbs": quant_bytes / (quant_ms * 1e-3) / 1e9,
