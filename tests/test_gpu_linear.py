@@ -1,9 +1,10 @@
 """GPU parity of the composed linear layer (qt2_linear_fwd / qt2_linear_bwd through the C ABI)
 against the oracle's fp64 results on the same seeded inputs.
 
-Small cases compare every output; the full-size case (the 1.9B-class layer: tokens 16384,
-d_in 2048, d_out 8192, the launch configuration the benchmark times) compares sampled rows
-that the oracle computes one by one, plus bit-exact codes and scales of those rows."""
+Small cases compare every output; the full-size cases (the 1.9B-class layer: tokens 16384,
+d_in 2048, d_out 8192, the launch configuration the benchmark times; the Llama-3-8B MLP gate/up
+4096 -> 14336 and down 14336 -> 4096 linears at 16384 tokens) compare sampled rows that the
+oracle computes one by one, plus bit-exact codes and scales of those rows."""
 import numpy as np
 import pytest
 import torch
@@ -80,11 +81,12 @@ def _view_rows(view: qt2.View, rows, R, C):
     return codes, scales, np.float32(view.tensor_scale.item())
 
 
-def test_full_size_llm1p9b_sampled():
-    """Tokens 16384, d_in 2048, d_out 8192: sampled rows of Y, dX and dW against the oracle, and
-    bit-exact codes/scales of the sampled rows of every quantized view."""
-    M, K, N = synth.SHAPES["llm1p9b"]
-    x, w, dy = synth.linear_inputs("llm1p9b", 0)
+@pytest.mark.parametrize("config", ["llm1p9b", "mlp8b_up", "mlp8b_down"])
+def test_full_size_sampled(config):
+    """Full-size layer: sampled rows of Y, dX and dW against the oracle, and bit-exact
+    codes/scales of the sampled rows of every quantized view."""
+    M, K, N = synth.SHAPES[config]
+    x, w, dy = synth.linear_inputs(config, 0)
     seed = 2024
     y, dx, dw = run_linear(x, w, dy, seed)
     rng = np.random.default_rng(0)
@@ -124,3 +126,5 @@ def test_full_size_llm1p9b_sampled():
     dw_ref = O.gemm(o_dy_col.dequant_rows(rows_n), o_x_col.dequant(), 2.0 ** -7)
     dw_g = dw[torch.from_numpy(rows_n).cuda()].cpu().numpy().astype(np.float64)
     assert _rel(dw_g, dw_ref) < 1e-5
+    _bound_check(dw_g, dw_ref, O.gemm(np.abs(o_dy_col.dequant_rows(rows_n)), np.abs(o_x_col.dequant()), 2.0 ** -7),
+                 False)
