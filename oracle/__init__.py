@@ -75,6 +75,8 @@ def lib():
                 "or_gemm_f64": (None, [vp, vp, i64, i64, i64, f64, i64, i64, vp]),
                 "or_rotated_amax_rows": (f32, [vp, i64, i64, vp, i64, i64]),
                 "or_sr_rows_dequant": (None, [vp, i64, i64, vp, f32, u64, u32, i64, i64, vp]),
+                "or_sr_tensor_scale": (f32, [f32]),
+                "or_sr_rows": (None, [vp, i64, i64, vp, f32, u64, u32, i64, i64, vp, vp]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -269,6 +271,29 @@ def sr_dequant(x, seed: int, tid: int, view: str = "row") -> np.ndarray:
     out = np.zeros((R, C), np.float64)
     _rows(lambda r0, r1: lib().or_sr_rows_dequant(_p(b), R, C, _p(sgn), A, seed, tid, r0, r1, _p(out)), R)
     return out
+
+
+def rotated_amax(b: np.ndarray, sgn: np.ndarray) -> np.float32:
+    """max |y| over a rotated view given as bf16 bits [R][C] (threads over row ranges; max is exact)."""
+    R, C = b.shape
+    parts = []
+    _rows(lambda r0, r1: parts.append(lib().or_rotated_amax_rows(_p(b), R, C, _p(sgn), r0, r1)), R)
+    return np.float32(max(parts))
+
+
+def sr(x, seed: int, tid: int, view: str = "row") -> View:
+    """Elementwise-SR NVFP4 view of the rotated tensor, every decision in binary32 (the GPU
+    SR baseline's contract): codes, canonical scales and the tensor scale g = A/2688."""
+    b = _bf16_bits(x)
+    if view == "col":
+        b = np.ascontiguousarray(b.T)
+    R, C = b.shape
+    sgn = rht_signs(seed)
+    A = rotated_amax(b, sgn)
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    _rows(lambda r0, r1: lib().or_sr_rows(_p(b), R, C, _p(sgn), A, seed, tid, r0, r1, _p(codes), _p(scales)), R)
+    return View(codes, scales, np.float32(lib().or_sr_tensor_scale(A)))
 
 
 def gemm(a: np.ndarray, b: np.ndarray, alpha: float = 1.0) -> np.ndarray:

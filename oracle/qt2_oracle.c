@@ -452,6 +452,68 @@ OR_EXPORT float or_rotated_amax_rows(const uint16_t *x, int64_t R, int64_t C, co
     return A;
 }
 
+/* The elementwise-SR quantizer of the rotated view as the GPU baseline computes it: every
+ * decision in binary32, so codes and scales are exactly reproducible ([QII-th] abstract and
+ * "fairness" answer: the SR-based TetraJet-v2 core, RHT along the inner dimension, is the
+ * baseline MS-EDEN is compared with; [QII-tg] "Method": SR rounds to one of the two grid
+ * neighbours with probability set by the distance).  Reading (the pages give no scale rule for
+ * the baseline): tensor scale g = A/2688 (A = max|y| over the view, 2688 = 6*448); the group
+ * scale is the smallest E4M3 value s with s >= a/(6g) (a = max|y| of the group, t = a/RN(6g)
+ * in binary32), so no element leaves the grid and SR stays unbiased; d = RN(s*g), r = RN(1/d),
+ * tq = min(|y|*r, 6); lo/hi = the E2M1 neighbours of tq; round up iff U < (tq-lo)/(hi-lo) with
+ * U = (u>>8)/2^24 and u = word e of the Philox stream (seed, tid), e = the element's canonical
+ * index r*C + c.  A view with A < 2^-100 is zero (g = 1); a group with a < 2^-100 gets scale 0
+ * and sign-only zero codes.  Codes keep the sign of y (a negative y that rounds to 0 is 0x8). */
+OR_EXPORT float or_sr_tensor_scale(float A) { return (A >= OR_TINY) ? A / 2688.0f : 1.0f; }
+
+OR_EXPORT void or_sr_rows(const uint16_t *x, int64_t R, int64_t C, const float sgn[128], float A, uint64_t seed,
+                          uint32_t tid, int64_t r0, int64_t r1, uint8_t *codes, uint8_t *scales)
+{
+    (void)R;
+    const float g = or_sr_tensor_scale(A);
+    const float g6 = 6.0f * g;
+    const int zero_view = !(A >= OR_TINY);
+    for (int64_t r = r0; r < r1; r++)
+        for (int64_t b = 0; b < C / 128; b++) {
+            float y[128];
+            for (int i = 0; i < 128; i++) y[i] = sgn[i] * or_bf16_to_f32(x[r * C + b * 128 + i]);
+            or_fwht128(y);
+            for (int q = 0; q < 8; q++) {
+                const int64_t j = b * 8 + q;   /* group index within the row */
+                float a = 0.0f;
+                for (int i = 0; i < 16; i++) if (fabsf(y[16 * q + i]) > a) a = fabsf(y[16 * q + i]);
+                uint8_t nib[16];
+                if (zero_view || !(a >= OR_TINY)) {
+                    scales[r * (C / 16) + j] = 0;
+                    for (int i = 0; i < 16; i++) nib[i] = signbit(y[16 * q + i]) ? 0x8 : 0x0;
+                } else {
+                    const float t = a / g6;
+                    int sc = 0;
+                    while (sc < 126 && or_e4m3_value((uint8_t)sc) < t) sc++;   /* ceil onto E4M3 */
+                    scales[r * (C / 16) + j] = (uint8_t)sc;
+                    const float d = or_e4m3_value((uint8_t)sc) * g;
+                    const float rr = 1.0f / d;
+                    for (int i = 0; i < 16; i++) {
+                        const float v = y[16 * q + i];
+                        float tq = fabsf(v) * rr;
+                        if (tq > 6.0f) tq = 6.0f;
+                        int lo = 0;
+                        for (int m = 1; m < 8; m++) if (OR_E2M1_MAG[m] <= tq) lo = m;
+                        if (lo < 7) {
+                            const float frac = (tq - OR_E2M1_MAG[lo]) / (OR_E2M1_MAG[lo + 1] - OR_E2M1_MAG[lo]);
+                            const uint32_t u = or_philox_word(seed, tid, (uint64_t)(r * C + 16 * j + i));
+                            const float U = (float)(u >> 8) * (1.0f / 16777216.0f);
+                            if (U < frac) lo++;
+                        }
+                        nib[i] = (uint8_t)((signbit(v) ? 0x8 : 0x0) | lo);
+                    }
+                }
+                for (int i = 0; i < 8; i++)
+                    codes[r * (C / 2) + j * 8 + i] = (uint8_t)(nib[2 * i] | (nib[2 * i + 1] << 4));
+            }
+        }
+}
+
 /* Plain NVFP4 with elementwise stochastic rounding, in the rotated domain -- the unbiased but
  * noisier estimator the pages compare MS-EDEN against ([QII-th] abstract; [QII-tg] "Method":
  * SR rounds up or down with probability set by the distance to the two neighbouring grid
