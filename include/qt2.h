@@ -129,6 +129,29 @@ QT2_API qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t co
                             size_t ws_bytes, qt2_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Backward quantizer with elementwise stochastic rounding: the baseline the Quartet II pages
+ * compare MS-EDEN against ([QII-th] abstract and the "fairness of the comparison" answer: the
+ * GPU-feasible TetraJet-v2 core, RHT along the inner dimension with stochastic rounding;
+ * [QII-tg] "Method": SR rounds to one of the two neighbouring grid points with probability set
+ * by the distance).  Same arguments, views and rotation as qt2_quant_msedEN; per view:
+ *   g = A/2688 (A = max|y| over the rotated view; A < 2^-100 gives a zero view with g = 1);
+ *   group scale = the smallest E4M3 value >= a/RN(6g) (a = max|y| of the group), so no element
+ *   leaves the grid and the estimate stays unbiased (the pages give no scale rule for the
+ *   baseline; this is the library's reading); d = RN(scale*g), r = RN(1/d);
+ *   element code = sign(y) | the E2M1 neighbour of min(|y|*r, 6) picked by stochastic
+ *   rounding with U = (u>>8)/2^24, u = word e of Philox(seed, tensor_id of the view), e = the
+ *   element's canonical index r*C + c in the view; a group with a < 2^-100 gets scale 0.
+ * Two passes over x (the max of the rotated view, then the quantization): the codes depend on
+ * the tensor scale.  Bit-identical to the reference algorithm for the same seed and ids.
+ * Workspace: at least qt2_quant_sr_workspace_size() bytes, 256-byte aligned (the view maxima).
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_sr_workspace_size(int64_t rows, int64_t cols, int layout_mask, size_t *bytes);
+QT2_API qt2_status qt2_quant_sr(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
+                                uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
+                                const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                                size_t ws_bytes, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * MS-EDEN without a workspace.  The Quartet II pages have no counterpart to this call; it is a
  * convenience of this library for callers that cannot allocate device memory for scratch (a
  * runtime that has handed all device memory to its own pools, a latency-critical path that

@@ -102,8 +102,7 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
 // Out: cw[2g], cw[2g+1] = codes of local group g (element 8w+i of the group in nibble i of
 // word w); Pq[g] = S * p of local group g.  Local groups 0, 1, 2, 3 are the block's groups 2h,
 // 2h+1, 4+2h, 5+2h.  amax = running max |y|.
-__device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint64_t nsg, uint32_t (&cw)[8],
-                                            float (&Pq)[4], float &amax) {
+__device__ __forceinline__ void rotate_tail(uint64_t (&P)[32], uint64_t sg, uint64_t nsg) {
     // strides 2, 4, 8, 16: slots j and j + hp of the same 16-slot half, same order on both threads
 #pragma unroll
     for (int hp = 1; hp < 16; hp <<= 1) {
@@ -132,6 +131,11 @@ __device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint
         P[k] = f2_add(keep, recv);                        // y[i] = z[i] + z[i + 64]
         P[16 + k] = f2_fma(sg, keep, f2_mul(recv, nsg));  // y[i + 64] = z[i] - z[i + 64]
     }
+}
+
+__device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint64_t nsg, uint32_t (&cw)[8],
+                                            float (&Pq)[4], float &amax) {
+    rotate_tail(P, sg, nsg);
 
     float nq[4], ptq[4], pq[4];
 #pragma unroll
@@ -198,6 +202,70 @@ __device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint
     for (int g = 0; g < 4; ++g) Pq[g] = __fmul_rn(S, pq[g]);
 }
 
+// Elementwise-SR quantization of the thread's four local groups after rotate_tail: the GPU
+// baseline of the pages' comparison ([QII-th] "fairness" answer: the TetraJet-v2 core, RHT
+// along the inner dimension with stochastic rounding; [QII-tg] "Method").  Every decision is one
+// binary32 operation: group scale code = the smallest E4M3 value >= a/(6g) (RNE, then one step
+// up if RNE fell below), d = RN(s*g), r = RN(1/d), tq = min(|y|*r, 6); tq's lower E2M1 neighbour
+// keeps the bits down to the top mantissa bit (the grid points of [2^k, 2^(k+1)) are 2^k and
+// 1.5*2^k for k >= 0; 0.5 and 0 below 1); the spacing to the upper neighbour is a power of two,
+// so frac = (tq - lo)/spacing is exact; round up iff (u>>8)*2^-24 < frac with u = Philox word e
+// of (seed, tid).  e_base[g] = canonical index of local group g's first element.
+__device__ __forceinline__ void sr_vector(const uint64_t (&P)[32], float g, float g6, bool zero_view, uint64_t seed,
+                                          uint32_t tid, const int64_t (&e_base)[4], uint32_t (&cw)[8],
+                                          uint32_t (&sc)[4], float &amax) {
+#pragma unroll
+    for (int gq = 0; gq < 4; ++gq) {
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f2_split(P[8 * gq + i], y[2 * i], y[2 * i + 1]);
+        const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
+        const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
+        const float m4 = absmax3(y[12], y[13], y[14]);
+        const float a = fmaxf(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+        amax = fmaxf(amax, a);
+        float q[16];
+        if (zero_view || !(a >= kTiny)) {
+            sc[gq] = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(y[i], 0.0f);   // sign-preserving zeros
+        } else {
+            const float t = __fdiv_rn(a, g6);
+            uint32_t c = e4m3_rne(t);
+            if (c < 126u && e4m3_value(c) < t) ++c;                        // ceil onto E4M3
+            sc[gq] = c;
+            const float d = __fmul_rn(e4m3_value(c), g);
+            const float r = __frcp_rn(d);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 u4 = philox_block(seed, tid, (uint64_t)((e_base[gq] >> 2) + k));
+                const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const int i = 4 * k + i2;
+                    const float tq = fminf(__fmul_rn(fabsf(y[i]), r), 6.0f);
+                    const uint32_t b = __float_as_uint(tq), e = b >> 23;
+                    const bool ge1 = e >= 127u;
+                    const float lo = __uint_as_float(ge1 ? (b & 0xFFC00000u) : (e == 126u ? 0x3F000000u : 0u));
+                    const float sp = __uint_as_float(ge1 ? (e - 1u) << 23 : 0x3F000000u);       // spacing
+                    const float inv = __uint_as_float(ge1 ? (255u - e) << 23 : 0x40000000u);     // 1/spacing
+                    const float frac = __fmul_rn(__fsub_rn(tq, lo), inv);
+                    const float U = __fmul_rn(__uint2float_rn(uw[i2] >> 8), 5.9604644775390625e-8f);   // 2^-24
+                    const float vq = (U < frac) ? __fadd_rn(lo, sp) : lo;
+                    q[i] = __uint_as_float(__float_as_uint(vq) | (__float_as_uint(y[i]) & 0x80000000u));
+                }
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float vh[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) vh[i] = q[8 * hh + i];
+            cw[2 * gq + hh] = e2m1x8(vh);   // exact: every value is a signed grid point
+        }
+    }
+}
+
 // Codes of the thread's groups {2h, 2h+1} and {4+2h, 5+2h} of a 128-block starting at group j0
 // of view row vr (codes_row points at the block's first code byte); pre-scales in tensor-core
 // scale order.
@@ -209,11 +277,24 @@ __device__ __forceinline__ void msed_store(uint8_t *codes_row, float *P_base, in
     *reinterpret_cast<float2 *>(P_base + sf_offset(vr, j0 + 4 + 2 * h, VC)) = make_float2(Pq[2], Pq[3]);
 }
 
-template <bool DO_ROW, bool DO_COL>
+// What one launch of the rotation producer emits per view (row view: [R][C]; column view: the
+// transpose [C][R]).
+struct RotViews {
+    uint8_t *row_codes, *col_codes;     // MS-EDEN and SR codes
+    float *row_P, *col_P;               // MS-EDEN fp32 pre-scales
+    uint8_t *row_scales, *col_scales;   // SR E4M3 scales
+    uint32_t *row_amax, *col_amax;      // max |y|: merged (MS-EDEN, max pass) or read (SR)
+    float *row_g, *col_g;               // SR tensor scales, written
+    uint32_t tid_row, tid_col;          // SR Philox tensor ids
+};
+enum RotMode { kModeEden = 0, kModeMax = 1, kModeSr = 2 };
+
+template <int MODE, bool DO_ROW, bool DO_COL>
 __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
-    msed_kernel(const __grid_constant__ CUtensorMap tmap, int64_t R, int64_t C, uint64_t seed,
-                uint8_t *__restrict__ row_codes, float *__restrict__ row_P, uint32_t *__restrict__ row_amax,
-                uint8_t *__restrict__ col_codes, float *__restrict__ col_P, uint32_t *__restrict__ col_amax) {
+    msed_kernel(const __grid_constant__ CUtensorMap tmap, int64_t R, int64_t C, uint64_t seed, RotViews out) {
+    uint8_t *const row_codes = out.row_codes, *const col_codes = out.col_codes;
+    float *const row_P = out.row_P, *const col_P = out.col_P;
+    uint32_t *const row_amax = out.row_amax, *const col_amax = out.col_amax;
     using Cfg = MsedCfg;
     constexpr int NS = Cfg::kStages;
     constexpr bool kBoth = DO_ROW && DO_COL;
@@ -261,6 +342,25 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     if (t == 0)
         for (int64_t i = 0; i < NS && i < my_tiles; ++i) issue(i);
 
+    // SR: tensor scale g = A/2688 of each view from its max pass; a view with A < 2^-100 is zero
+    float g_r = 1.0f, g6_r = 6.0f, g_c = 1.0f, g6_c = 6.0f;
+    bool zero_r = true, zero_c = true;
+    if constexpr (MODE == kModeSr) {
+        if (DO_ROW) {
+            const float A = __uint_as_float(*row_amax);
+            zero_r = !(A >= kTiny);
+            g_r = zero_r ? 1.0f : __fdiv_rn(A, 2688.0f);
+            g6_r = __fmul_rn(6.0f, g_r);
+            if (blockIdx.x == 0 && t == 0) *out.row_g = g_r;
+        }
+        if (DO_COL) {
+            const float A = __uint_as_float(*col_amax);
+            zero_c = !(A >= kTiny);
+            g_c = zero_c ? 1.0f : __fdiv_rn(A, 2688.0f);
+            g6_c = __fmul_rn(6.0f, g_c);
+            if (blockIdx.x == 0 && t == 0) *out.col_g = g_c;
+        }
+    }
     const float sigma = h ? -1.0f : 1.0f;
     const uint64_t sg = f2(sigma, sigma), nsg = f2(-sigma, -sigma);
     const bool rows = kBoth ? team == 0 : DO_ROW;
@@ -330,19 +430,42 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             const uint32_t old = atomicAdd(&done_cnt[s], 1u);
             if (old == (uint32_t)(i / NS + 1) * kConsumers - 1 && i + NS < my_tiles) issue(i + NS);
         }
-        uint32_t cw[8];
-        float Pq[4];
-        msed_vector(P, sg, nsg, cw, Pq, amax);
-        if (rows) {
-            const int64_t vr = r0 + u;
-            msed_store(row_codes + vr * (C >> 1) + (c0 >> 1), row_P, vr, c0 >> 4, C, h, cw, Pq);
+        const int64_t vr = rows ? r0 + u : c0 + u;   // view row (the column view is [C][R])
+        const int64_t VC = rows ? C : R, b0 = rows ? c0 : r0;   // view row length, block start
+        uint8_t *const vcodes = (rows ? row_codes : col_codes) + vr * (VC >> 1) + (b0 >> 1);
+        if constexpr (MODE == kModeEden) {
+            uint32_t cw[8];
+            float Pq[4];
+            msed_vector(P, sg, nsg, cw, Pq, amax);
+            msed_store(vcodes, rows ? row_P : col_P, vr, b0 >> 4, VC, h, cw, Pq);
+        } else if constexpr (MODE == kModeMax) {
+            rotate_tail(P, sg, nsg);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                float y0, y1;
+                f2_split(P[k], y0, y1);
+                amax = absmax3(amax, y0, y1);
+            }
         } else {
-            const int64_t vr = c0 + u;   // row of the transposed view [C][R]
-            msed_store(col_codes + vr * (R >> 1) + (r0 >> 1), col_P, vr, r0 >> 4, R, h, cw, Pq);
+            rotate_tail(P, sg, nsg);
+            // local groups 0, 1, 2, 3 are the block's groups 2h, 2h+1, 4+2h, 5+2h
+            const int64_t e0 = vr * VC + b0;
+            const int64_t e_base[4] = {e0 + 32 * h, e0 + 32 * h + 16, e0 + 64 + 32 * h, e0 + 80 + 32 * h};
+            uint32_t cw[8], scq[4];
+            sr_vector(P, rows ? g_r : g_c, rows ? g6_r : g6_c, rows ? zero_r : zero_c, seed,
+                      rows ? out.tid_row : out.tid_col, e_base, cw, scq, amax);
+            *reinterpret_cast<uint4 *>(vcodes + 16 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint4 *>(vcodes + 32 + 16 * h) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            uint8_t *const sb = rows ? out.row_scales : out.col_scales;
+            *reinterpret_cast<uint16_t *>(sb + sf_offset(vr, (b0 >> 4) + 2 * h, VC)) = (uint16_t)(scq[0] | (scq[1] << 8));
+            *reinterpret_cast<uint16_t *>(sb + sf_offset(vr, (b0 >> 4) + 4 + 2 * h, VC)) =
+                (uint16_t)(scq[2] | (scq[3] << 8));
         }
     }
-    const uint32_t bm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
-    if (lane == 0 && bm != 0) atomicMax(rows ? row_amax : col_amax, bm);
+    if constexpr (MODE != kModeSr) {
+        const uint32_t bm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
+        if (lane == 0 && bm != 0) atomicMax(rows ? row_amax : col_amax, bm);
+    }
     __syncthreads();
     if (t == 0) {
         // Only after a timeout can a load still be in flight: wait (bounded) for each stage's last one.

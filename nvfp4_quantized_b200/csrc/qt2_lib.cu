@@ -53,14 +53,13 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaGetLastError();
 }
 
-template <bool ROW, bool COL>
-static cudaError_t launch_msed_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed, DevView row,
-                                       DevView col, float *P_row, float *P_col, uint32_t *amax_row,
-                                       uint32_t *amax_col, cudaStream_t s) {
+template <int MODE, bool ROW, bool COL>
+static cudaError_t launch_rot_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed,
+                                      const RotViews &out, cudaStream_t s) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(msed_kernel<ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(msed_kernel<MODE, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         MsedCfg::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -68,19 +67,29 @@ static cudaError_t launch_msed_variant(const CUtensorMap &tmap, int64_t R, int64
     // one CTA per SM; a single view needs two tiles per CTA to keep both halves busy
     const int64_t per_cta = (ROW && COL) ? 1 : 2;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((ntiles + per_cta - 1) / per_cta, sm_count()));
-    msed_kernel<ROW, COL><<<(unsigned)grid, MsedCfg::kThreads, MsedCfg::kSmemBytes, s>>>(
-        tmap, R, C, seed, row.codes, P_row, amax_row, col.codes, P_col, amax_col);
+    msed_kernel<MODE, ROW, COL><<<(unsigned)grid, MsedCfg::kThreads, MsedCfg::kSmemBytes, s>>>(tmap, R, C, seed, out);
     return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_rot(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col, uint64_t seed,
+                              const RotViews &out, cudaStream_t s) {
+    if (do_row && do_col) return launch_rot_variant<MODE, true, true>(tmap, R, C, seed, out, s);
+    if (do_row) return launch_rot_variant<MODE, true, false>(tmap, R, C, seed, out, s);
+    return launch_rot_variant<MODE, false, true>(tmap, R, C, seed, out, s);
 }
 
 cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col,
                               uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
                               uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s) {
-    if (do_row && do_col)
-        return launch_msed_variant<true, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
-    if (do_row)
-        return launch_msed_variant<true, false>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
-    return launch_msed_variant<false, true>(tmap, R, C, seed, row, col, P_row, P_col, amax_row, amax_col, s);
+    RotViews out{};
+    out.row_codes = row.codes;
+    out.col_codes = col.codes;
+    out.row_P = P_row;
+    out.col_P = P_col;
+    out.row_amax = amax_row;
+    out.col_amax = amax_col;
+    return launch_rot<kModeEden>(tmap, R, C, do_row, do_col, seed, out, s);
 }
 
 cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
@@ -367,6 +376,39 @@ size_t msed_scratch_bytes(int64_t rows, int64_t cols, int layout_mask) {
 
 qt2_status msed_device_check() { return check_device(); }
 
+// Elementwise-SR view(s) of the rotated tensor: a max pass over the rotated view(s), then the
+// quantize pass (the SR scales need the tensor scale first).
+size_t sr_ws(uint32_t **amax, void *ws) {
+    Carve c(ws);
+    *amax = reinterpret_cast<uint32_t *>(c.take(2 * sizeof(uint32_t)));
+    return c.used;
+}
+qt2_status sr_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, int mask, uint64_t seed, uint32_t tid_row,
+                      uint32_t tid_col, DevView row, DevView col, uint32_t *amax, cudaStream_t s) {
+    CUtensorMap tmap;
+    if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
+                        128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return QT2_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    const bool do_row = (mask & QT2_LAYOUT_ROW) != 0, do_col = (mask & QT2_LAYOUT_COL) != 0;
+    RotViews out{};
+    out.row_codes = row.codes;
+    out.col_codes = col.codes;
+    out.row_scales = row.scales;
+    out.col_scales = col.scales;
+    out.row_amax = amax;
+    out.col_amax = amax + 1;
+    out.row_g = row.tensor_scale;
+    out.col_g = col.tensor_scale;
+    out.tid_row = tid_row;
+    out.tid_col = tid_col;
+    e = launch_rot<kModeMax>(tmap, rows, cols, do_row, do_col, seed, out, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_rot<kModeSr>(tmap, rows, cols, do_row, do_col, seed, out, s);
+    return from_cuda(e);
+}
+
 qt2_status msed_enqueue_on_scratch(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
                                    uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
                                    const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *scratch,
@@ -464,6 +506,34 @@ qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t cols, int6
                         (layout_mask & QT2_LAYOUT_ROW) ? dev_view(row_out) : none,
                         (layout_mask & QT2_LAYOUT_COL) ? dev_view(col_out) : none, P_row, P_col, amax,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+qt2_status qt2_quant_sr_workspace_size(int64_t rows, int64_t cols, int layout_mask, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols)) return QT2_ERR_SHAPE;
+    uint32_t *a;
+    *bytes = sr_ws(&a, nullptr);
+    return QT2_OK;
+}
+qt2_status qt2_quant_sr(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask, uint64_t seed,
+                        uint32_t tensor_id_row, uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
+                        const qt2_nvfp4_view *col_out, void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_ROW) && !view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if ((layout_mask & QT2_LAYOUT_COL) && !view_ok(col_out)) return col_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    uint32_t *amax;
+    if (ws_bytes < sr_ws(&amax, workspace)) return QT2_ERR_WORKSPACE;
+    if ((st = check_device()) != QT2_OK) return st;
+    const DevView none{nullptr, nullptr, nullptr};
+    return sr_enqueue(x_bf16, rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
+                      (layout_mask & QT2_LAYOUT_ROW) ? dev_view(row_out) : none,
+                      (layout_mask & QT2_LAYOUT_COL) ? dev_view(col_out) : none, amax,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 qt2_status qt2_gemm_nvfp4(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,

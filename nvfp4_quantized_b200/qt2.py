@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
                 "qt2_quant_msedEN_workspace_size": (i32, [i64, i64, i32, psz]),
                 "qt2_quant_msedEN": (i32, [vp, i64, i64, i64, i32, u64, u32, u32, pv, pv, vp, sz, vp]),
                 "qt2_quant_msedEN_noalloc": (i32, [vp, i64, i64, i64, i32, u64, u32, u32, pv, pv, vp]),
+                "qt2_quant_sr_workspace_size": (i32, [i64, i64, i32, psz]),
+                "qt2_quant_sr": (i32, [vp, i64, i64, i64, i32, u64, u32, u32, pv, pv, vp, sz, vp]),
                 "qt2_gemm_nvfp4": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_linear_fwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_fwd": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
@@ -199,6 +201,22 @@ def qt2_quant_msedEN_noalloc(x: torch.Tensor, rows: int, cols: int, ld: int, lay
     _check("qt2_quant_msedEN_noalloc", lib().qt2_quant_msedEN_noalloc(
         _ptr(x), rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
         ctypes.byref(r) if r else None, ctypes.byref(c) if c else None, _stream(stream)))
+
+
+def qt2_quant_sr_workspace_size(rows: int, cols: int, layout_mask: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qt2_quant_sr_workspace_size", lib().qt2_quant_sr_workspace_size(rows, cols, layout_mask, ctypes.byref(n)))
+    return n.value
+
+
+def qt2_quant_sr(x: torch.Tensor, rows: int, cols: int, ld: int, layout_mask: int, seed: int, tensor_id_row: int,
+                 tensor_id_col: int, row_out: View | None, col_out: View | None, workspace: torch.Tensor,
+                 ws_bytes: int, stream=None) -> None:
+    r = row_out.c() if row_out is not None else None
+    c = col_out.c() if col_out is not None else None
+    _check("qt2_quant_sr", lib().qt2_quant_sr(
+        _ptr(x), rows, cols, ld, layout_mask, seed, tensor_id_row, tensor_id_col,
+        ctypes.byref(r) if r else None, ctypes.byref(c) if c else None, _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def qt2_gemm_nvfp4(a: View, b: View, M: int, N: int, K: int, alpha: float, c: torch.Tensor, c_dtype: int,
