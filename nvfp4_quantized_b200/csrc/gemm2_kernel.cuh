@@ -44,9 +44,9 @@
 //                        block-scaled MMA reads), then commits to "sftm" of region j % 5 and to
 //                        "sf_free" of the scale slot on both SMs.
 //   warps 4..11        : epilogue.  Warp w reads TMEM lane quadrant w%4, columns [0, 128) for
-//                        warps 4..7 and [128, 256) for warps 8..11, in 32-column chunks, scales
-//                        them and stores its rows straight to global memory (bf16 or fp32); the
-//                        accumulator is released right after its last tensor-memory read.
+//                        warps 4..7 and [128, 256) for warps 8..11, all into registers, releases
+//                        the accumulator, then scales and stores its rows straight to global
+//                        memory (bf16 or fp32) while the next tile's MMAs run.
 // Tensor memory: accumulator columns [0, 256); scale region r (of stage j, r = j % 5) at
 // 256 + 48 r (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
 // Every wait is bounded; on a timeout the CTA records QT2_ERR_TIMEOUT, the leader drains the
@@ -341,34 +341,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             const int64_t row = (int64_t)pm * 256 + rank * 128 + quad * 32 + lane;
             const int64_t col = (int64_t)pn * 256 + cb;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + cb;
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                tmem_ld_32x32b_x16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                tmem_ld_wait();
-                if (c == 96) {   // last read of this tile: release the accumulator
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(acc_empty_leader);
-                }
-                if (c_dtype == QT2_DTYPE_F32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + row * ldc + col + c);
+            // All 128 columns into registers first, then release the accumulator, so the next
+            // tile's MMAs overlap the scaling and the stores.
+            uint32_t v[128];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
-                                             __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc);
-                } else {
-                    uint32_t p[16];
+            for (int c = 0; c < 128; c += 16)
+                tmem_ld_32x32b_x16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            if (c_dtype == QT2_DTYPE_F32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + row * ldc + col);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]) * sc,
-                                                                  __uint_as_float(v[2 * i + 1]) * sc);
-                        p[i] = *reinterpret_cast<uint32_t *>(&b2);
+                for (int i = 0; i < 32; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
+                                         __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc);
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(Cout) + row * ldc + col);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    uint32_t p[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2 * k]) * sc,
+                                                                  __uint_as_float(v[8 * i + 2 * k + 1]) * sc);
+                        p[k] = *reinterpret_cast<uint32_t *>(&b2);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(Cout) + row * ldc + col + c);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+                    dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
                 }
             }
         }
