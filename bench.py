@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "Quartet II linear fwd+bwd TFLOPS; quantizer GB/s; % of FP4/HBM roofline"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 14   # amax x2, fwd46 x2, gemm x3, MS-EDEN tiles x3, scale finalize x4
+KERNELS_PER_STEP = 13   # per step: 2 max + 2 fwd46 + 3 GEMM + 3 MS-EDEN producers + 3 finalize (dY views share one)
 
 # Algorithmic bytes per input element of each quantizer call (reads + writes the method needs).
 BYTES_FWD46 = 2 + 2 + 0.5 + 1 / 16            # max pass read, quantize read, codes, scales

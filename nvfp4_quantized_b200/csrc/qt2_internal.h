@@ -32,8 +32,9 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
 cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col,
                               uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
                               uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s);
-cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
-                                 uint32_t tid, DevView out, cudaStream_t s);
+cudaError_t launch_msed_finalize(const float *P_a, int64_t R_a, int64_t C_a, const uint32_t *amax_a, uint32_t tid_a,
+                                 DevView out_a, const float *P_b, int64_t R_b, int64_t C_b, const uint32_t *amax_b,
+                                 uint32_t tid_b, DevView out_b, uint64_t seed, cudaStream_t s);
 cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
                               int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s);
 

@@ -92,13 +92,24 @@ cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, boo
     return launch_rot<kModeEden>(tmap, R, C, do_row, do_col, seed, out, s);
 }
 
-cudaError_t launch_msed_finalize(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint64_t seed,
-                                 uint32_t tid, DevView out, cudaStream_t s) {
+static FinalizeJob finalize_job(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint32_t tid,
+                                DevView out, int64_t max_blocks) {
     const int64_t words = (R * C) >> 6;
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((words + 255) / 256, (int64_t)sm_count() * 16));
-    msed_finalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(P), R, C, amax_word, seed,
-                                                          tid, reinterpret_cast<uint32_t *>(out.scales),
-                                                          out.tensor_scale);
+    FinalizeJob j{reinterpret_cast<const float4 *>(P), R, C, amax_word, tid,
+                  reinterpret_cast<uint32_t *>(out.scales), out.tensor_scale, 0};
+    j.blocks = std::max<int64_t>(1, std::min<int64_t>((words + 255) / 256, max_blocks));
+    return j;
+}
+
+// Finalize one view, or two in one launch when `P_b` is given (the grid is split by size).
+cudaError_t launch_msed_finalize(const float *P_a, int64_t R_a, int64_t C_a, const uint32_t *amax_a, uint32_t tid_a,
+                                 DevView out_a, const float *P_b, int64_t R_b, int64_t C_b, const uint32_t *amax_b,
+                                 uint32_t tid_b, DevView out_b, uint64_t seed, cudaStream_t s) {
+    const int64_t cap = (int64_t)sm_count() * 16;
+    FinalizeJob ja = finalize_job(P_a, R_a, C_a, amax_a, tid_a, out_a, P_b ? cap / 2 : cap);
+    FinalizeJob jb = P_b ? finalize_job(P_b, R_b, C_b, amax_b, tid_b, out_b, cap / 2) : ja;
+    const int64_t blocks = ja.blocks + (P_b ? jb.blocks : 0);
+    msed_finalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(ja, jb, seed);
     return cudaGetLastError();
 }
 
@@ -268,15 +279,14 @@ qt2_status msed_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, i
     e = launch_msed_tiles(tmap, rows, cols, (mask & QT2_LAYOUT_ROW) != 0, (mask & QT2_LAYOUT_COL) != 0, seed, row, col,
                           P_row, P_col, amax, amax + 1, s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
-    if (mask & QT2_LAYOUT_ROW) {
-        e = launch_msed_finalize(P_row, rows, cols, amax, seed, tid_row, row, s);
-        if (e != cudaSuccess) return QT2_ERR_CUDA;
-    }
-    if (mask & QT2_LAYOUT_COL) {
-        e = launch_msed_finalize(P_col, cols, rows, amax + 1, seed, tid_col, col, s);
-        if (e != cudaSuccess) return QT2_ERR_CUDA;
-    }
-    return QT2_OK;
+    if ((mask & QT2_LAYOUT_ROW) && (mask & QT2_LAYOUT_COL))
+        e = launch_msed_finalize(P_row, rows, cols, amax, tid_row, row, P_col, cols, rows, amax + 1, tid_col, col,
+                                 seed, s);
+    else if (mask & QT2_LAYOUT_ROW)
+        e = launch_msed_finalize(P_row, rows, cols, amax, tid_row, row, nullptr, 0, 0, nullptr, 0, row, seed, s);
+    else
+        e = launch_msed_finalize(P_col, cols, rows, amax + 1, tid_col, col, nullptr, 0, 0, nullptr, 0, col, seed, s);
+    return from_cuda(e);
 }
 
 qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *amax,

@@ -110,13 +110,15 @@ struct Fwd46Scale {
     uint64_t rr;       // (1/d, 1/d)
 };
 
-__device__ __forceinline__ Fwd46Scale fwd46_scale(float a, float g, float gk) {
+// d and 1/d depend on the scale code only (g is fixed per tensor): the block tabulates them once
+// for the 128 non-negative E4M3 codes (tab_d[c] = RN(val(c)*g), tab_r[c] = RN(1/tab_d[c]),
+// tab_r[0] = 0), so a candidate costs one division, one convert and two shared loads.
+__device__ __forceinline__ Fwd46Scale fwd46_scale(float a, float gk, const float *tab_d, const float *tab_r) {
     Fwd46Scale c;
     c.code = e4m3_rne(__fdiv_rn(a, gk));
-    const float d = __fmul_rn(e4m3_value(c.code), g);
-    const float r = (c.code == 0) ? 0.0f : __frcp_rn(d);
+    const float r = tab_r[c.code];
     c.rr = f2(r, r);
-    c.d = d;
+    c.d = tab_d[c.code];
     return c;
 }
 
@@ -156,13 +158,21 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
     const float g = zero_tensor ? 1.0f : __fdiv_rn(A, kFwd46Denominator);
     const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+    __shared__ float tab_d[128], tab_r[128];
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(e4m3_value(threadIdx.x), g);
+        tab_d[threadIdx.x] = d;
+        tab_r[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(d);
+    }
+    __syncthreads();
 
     const uint32_t G = (uint32_t)(C >> 4);                 // groups per row (a multiple of 8)
     const uint64_t total = (uint64_t)R * G;                // a multiple of 1024
+    const bool small = total <= 0xFFFFFFFFull;              // 32-bit index arithmetic suffices
     const int lane = threadIdx.x & 31;
     for (uint64_t gi = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < total;
          gi += (uint64_t)gridDim.x * blockDim.x) {
-        const uint64_t r = gi / G;
+        const uint64_t r = small ? (uint64_t)((uint32_t)gi / G) : gi / G;
         const uint32_t q = (uint32_t)(gi - r * G);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (uint64_t)q * 16);
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
             for (int i = 0; i < s / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
         }
         const float a = m8[0];
-        const Fwd46Scale s6 = fwd46_scale(a, g, g6), s4 = fwd46_scale(a, g, g4);
+        const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
         uint32_t c6[2], c4[2];
         float e6[8], e4[8];
         fwd46_candidate(X, s6, c6, e6);
@@ -222,22 +232,33 @@ __device__ __forceinline__ uint4 rotation_sign_words(uint64_t seed) { return phi
 // One thread per 4-group scale word; P is read in the same scale-factor order, so both the
 // 16-byte reads and the 4-byte writes are contiguous across a warp.
 // ---------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) msed_finalize_kernel(const float4 *__restrict__ P, int64_t VR, int64_t VC,
-                                                            const uint32_t *__restrict__ amax_word, uint64_t seed,
-                                                            uint32_t tid, uint32_t *__restrict__ scale_words,
-                                                            float *__restrict__ tensor_scale) {
-    const float A = __uint_as_float(*amax_word);
+struct FinalizeJob {
+    const float4 *P;            // pre-scales in scale-factor order
+    int64_t VR, VC;             // view shape
+    const uint32_t *amax_word;  // the view's max |y|
+    uint32_t tid;               // Philox tensor id of the view
+    uint32_t *scale_words;
+    float *tensor_scale;
+    int64_t blocks;             // blocks of the launch that serve this job
+};
+
+// One launch finalizes one or two views: blocks [0, j0.blocks) serve j0, the rest j1.
+__global__ void __launch_bounds__(256) msed_finalize_kernel(FinalizeJob j0, FinalizeJob j1, uint64_t seed) {
+    const bool second = (int64_t)blockIdx.x >= j0.blocks;
+    const FinalizeJob &jb = second ? j1 : j0;
+    const int64_t bid = second ? blockIdx.x - j0.blocks : blockIdx.x, nb = jb.blocks;
+    const float A = __uint_as_float(*jb.amax_word);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kMsedDenominator) : 1.0f;
     const float ginv = __frcp_rn(g);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-    const int64_t words = (VR * VC) >> 6;
-    const int64_t atoms_per_rowblock = VC >> 6;
-    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words; w += (int64_t)gridDim.x * blockDim.x) {
+    if (bid == 0 && threadIdx.x == 0) *jb.tensor_scale = g;
+    const int64_t words = (jb.VR * jb.VC) >> 6;
+    const int64_t atoms_per_rowblock = jb.VC >> 6;
+    for (int64_t w = bid * blockDim.x + threadIdx.x; w < words; w += nb * blockDim.x) {
         const int64_t atom = w >> 7, wi = w & 127;
         const int64_t r = (atom / atoms_per_rowblock) * 128 + (wi & 3) * 32 + (wi >> 2);
         const int64_t j4 = atom % atoms_per_rowblock;        // groups 4*j4 .. 4*j4+3 of view row r
-        const float4 p = __ldcs(P + w);
-        const uint4 u = philox_block(seed, tid, (uint64_t)(r * atoms_per_rowblock + j4));
+        const float4 p = __ldcs(jb.P + w);
+        const uint4 u = philox_block(seed, jb.tid, (uint64_t)(r * atoms_per_rowblock + j4));
         const float pv[4] = {p.x, p.y, p.z, p.w};
         const uint32_t uv[4] = {u.x, u.y, u.z, u.w};
         uint32_t word = 0;
@@ -247,7 +268,7 @@ __global__ void __launch_bounds__(256) msed_finalize_kernel(const float4 *__rest
             const uint32_t s = (v < kSrCutoff) ? e4m3_rne(v) : e4m3_sr(v, uv[k]);
             word |= s << (8 * k);
         }
-        scale_words[w] = word;
+        jb.scale_words[w] = word;
     }
 }
 
