@@ -30,6 +30,10 @@
 //   one view   : warps 0..7 and 8..15 take alternate tiles.
 // A ring stage is refilled by the last warp that has read it (a shared counter), so the two
 // halves of the CTA drift freely by up to the ring depth.
+//
+// The same producer serves the elementwise-SR baseline (qt2_quant_sr): kModeMax merges max |y|
+// of the rotated view(s) and writes nothing else; kModeSr then quantizes with that tensor scale
+// (sr_vector).  kModeEden is MS-EDEN.
 #pragma once
 
 #include "quant_kernels.cuh"
