@@ -10,48 +10,38 @@
 // per flop.  Operand loads are plain TMA loads (no multicast) whose completion both SMs report to
 // the leader SM's barrier.
 //
-// What bounds the pipeline on B200 (measured with timing-only variants of this kernel, dgrad
-// shape 16384 x 2048 x 8192): the MMA stream alone runs at ~7 PFLOP/s; the code loads alone
-// (5-stage ring, released by tcgen05.commit) stream ~12 TB/s into the SMs, because a TMA load
-// takes ~2 us under full load and the ring keeps ~190 KB in flight per SM.  What is left is the
-// scale path: the 12 tcgen05.cp of a stage cost ~33 ns each when the MMA thread issues them,
-// overlap the MMAs when another thread does, but then sit on the critical path between a
-// stage's MMAs retiring (its TMEM scale region) and the next use of that region; handing the
-// scales over through tcgen05.st from registers is slower still.  The best arrangement found:
-// the scales travel in their own deeper ring, two stages ahead of the codes, and a copier
-// thread moves them as soon as a region frees (~2.9 PFLOP/s on that shape, ~50% of a library
-// NVFP4 GEMM on the same GPU).
+// Issue discipline (measured on B200): every role that issues TMA or tcgen05 instructions runs
+// as a whole converged warp and lets one lane chosen by elect.sync issue them.  The operands
+// are then warp-uniform values the instructions take directly; issued from a lone lane of a
+// diverged warp each tcgen05.cp / tcgen05.mma / TMA load cost ~30 ns of issue overhead, which
+// made the 12 scale copies of a stage the bottleneck (the same kernel in that form ran the
+// layer's dgrad GEMM in 0.186 ms; converged, in 0.115 ms).
 //
 // Roles, per CTA of 384 threads (12 warps), persistent over 256x256 tiles (K = 256 per stage):
-//   warp 0, lanes 0..9 : code producers, one thread per operand and ring slot (TMA loads issued
-//                        by one thread are processed one after another).  Lane s loads A, lane
-//                        5 + s loads B of code slot s: own 128 rows of A and own 128 of the 256
-//                        B rows, reported to the leader's "full" barrier after the slot's
-//                        "empty" (the MMAs that read it) completed.
-//   warp 3, lanes 0..6 : scale producers (a warp of their own: lanes of one warp that wait on
-//                        different barriers slow each other down).  Lane q loads SFA and SFB of
-//                        scale slot q (A: own rows; B: all 256 rows, because each SM's tensor
-//                        memory needs the scales of every B column) into the leader's "sf_full"
-//                        after "sf_free" (the copies that read it) completed.
-//   warp 1             : allocates/frees 512 TMEM columns (both SMs); on the leader, one thread
-//                        issues the four 256x256x64 MMAs of each stage after "full" and "sftm"
-//                        and a tcgen05.commit that frees the code slot (and the stage's scale
-//                        region of TMEM) on both SMs.
-//   warp 2, leader     : scale copier.  For stage j: waits "sf_full" of scale slot j % 7 and the
-//                        MMAs of stage j - 5 (its TMEM scale region), copies the 12 scale atoms
-//                        from both SMs' shared memory into their tensor memory (tcgen05.cp
-//                        32x128b, replicated into the four lane quadrants, the layout the
-//                        block-scaled MMA reads), then commits to "sftm" of region j % 5 and to
-//                        "sf_free" of the scale slot on both SMs.
+//   warp 0             : producer.  Per stage, after "empty" (the MMAs that read the slot
+//                        completed), one lane loads the slot's own 128 rows of A, own 128 of the
+//                        256 B rows, the A scales of its rows and the B scales of all 256 rows
+//                        (each SM's tensor memory needs the scales of every B column): 38 KB,
+//                        reported to the leader's "full" barrier (the leader expects both SMs'
+//                        bytes).
+//   warp 2, leader     : scale copier.  After "full", copies the stage's 12 scale atoms from
+//                        both SMs' shared memory into their tensor memory (tcgen05.cp 32x128b,
+//                        replicated into the four lane quadrants, the layout the block-scaled
+//                        MMA reads) and commits to "sftm".  The stage's scale region is free by
+//                        then: its data could only land after the MMAs of the stage that last
+//                        used the region completed.
+//   warp 1             : allocates/frees 512 TMEM columns (both SMs); on the leader, after
+//                        "full" and "sftm", issues the four 256x256x64 MMAs of the stage and a
+//                        tcgen05.commit that frees the slot on both SMs ("empty").
 //   warps 4..11        : epilogue.  Warp w reads TMEM lane quadrant w%4, columns [0, 128) for
 //                        warps 4..7 and [128, 256) for warps 8..11, all into registers, releases
 //                        the accumulator, then scales and stores its rows straight to global
 //                        memory (bf16 or fp32) while the next tile's MMAs run.
-// Tensor memory: accumulator columns [0, 256); scale region r (of stage j, r = j % 5) at
-// 256 + 48 r (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
+// Tensor memory: accumulator columns [0, 256); scale region s (of ring slot s) at 256 + 48 s
+// (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
 // Every wait is bounded; on a timeout the CTA records QT2_ERR_TIMEOUT, the leader drains the
-// loads and tensor-core work that were issued, both CTAs meet at the final cluster barrier and
-// free TMEM.
+// loads (of both SMs) and tensor-core work that were issued, both CTAs meet at the final cluster
+// barrier and free TMEM.
 #pragma once
 
 #include "qt2_device.cuh"
@@ -153,10 +143,16 @@ __device__ __forceinline__ void tc_commit_pair_leader(uint32_t bar) {
                  : "memory");
 }
 
+// One lane of a converged warp (PTX elect.sync).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xFFFFFFFF;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(p));
+    return p != 0;
+}
+
 // ------------------------------------------------------------------ configuration
 struct Gemm2Cfg {
-    static constexpr int kStages = 5;             // code ring (A + B)
-    static constexpr int kSfStages = 7;           // scale ring, loaded up to 2 stages ahead
+    static constexpr int kStages = 5;             // ring of A + B codes and their scales
     static constexpr int kThreads = 384;
     static constexpr int kEpiWarp0 = 4;
     static constexpr int kEpiWarps = 8;
@@ -164,15 +160,14 @@ struct Gemm2Cfg {
     static constexpr int kB = 128 * 128;          // own half of the 256 B rows
     static constexpr int kSfa = 4 * 512;          // 4 k-blocks x one 512-byte atom
     static constexpr int kSfb = 2 * 4 * 512;      // both 128-row atoms of B, 4 k-blocks each
-    static constexpr int kStageBytes = kA + kB;   // 32 KB, keeps 1 KB alignment
-    static constexpr int kSfStageBytes = kSfa + kSfb;
-    static constexpr int kSmemBytes = kStages * kStageBytes + kSfStages * kSfStageBytes + 1024 + 512;
+    static constexpr int kStageBytes = kA + kB + kSfa + kSfb;   // 38 KB, keeps 1 KB alignment
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
     static constexpr int kTmemCols = 512;         // accumulator 256 + 5 scale regions x 48
     static constexpr int kSfRegionCols = 48;
     // E2M1 x E2M1, UE4M3 scales, K-major A and B, M = 256 (pair), N = 256
     static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (32u << 17) | (16u << 24);
 };
-static_assert(Gemm2Cfg::kStages * 2 <= 32 && Gemm2Cfg::kSfStages <= 32, "producer lanes");
+static_assert(Gemm2Cfg::kStageBytes % 1024 == 0, "stage alignment");
 static_assert(256 + Gemm2Cfg::kStages * Gemm2Cfg::kSfRegionCols <= Gemm2Cfg::kTmemCols, "TMEM columns");
 
 
@@ -182,14 +177,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                            const float *__restrict__ gA, const float *__restrict__ gB, float alpha,
                            void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype) {
     using Cfg = Gemm2Cfg;
-    constexpr int S = Cfg::kStages, SF = Cfg::kSfStages;
+    constexpr int S = Cfg::kStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint8_t *sf_base = base + S * Cfg::kStageBytes;
-    // barriers: full[S] sftm[S] empty[S] sf_full[SF] sf_free[SF] acc_full acc_empty
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sf_base + SF * Cfg::kSfStageBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 2 * SF + 2);
-    int *consumed_slot = reinterpret_cast<int *>(tmem_slot + 1);
+    // barriers: full[S] sftm[S] empty[S] acc_full acc_empty
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + S * Cfg::kStageBytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 2);
 
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -200,19 +193,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     const int my_tiles = tiles > cluster_id ? (tiles - 1 - cluster_id) / num_clusters + 1 : 0;
     const int total = my_tiles * nks;   // stages this pair runs
     const uint32_t full0 = smem_u32(bars), sftm0 = smem_u32(bars + S), empty0 = smem_u32(bars + 2 * S);
-    const uint32_t sf_full0 = smem_u32(bars + 3 * S), sf_free0 = smem_u32(bars + 3 * S + SF);
-    const uint32_t acc_full = smem_u32(bars + 3 * S + 2 * SF), acc_empty = acc_full + 8;
+    const uint32_t acc_full = smem_u32(bars + 3 * S), acc_empty = acc_full + 8;
 
     if (threadIdx.x == 0) {
-        *consumed_slot = 0;
         for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8 * s, 2);    // the A and B issuers of the leader
+            mbar_init(full0 + 8 * s, 1);    // the leader's producer (expects both SMs' bytes)
             mbar_init(sftm0 + 8 * s, 1);    // the scale copier's commit
-            mbar_init(empty0 + 8 * s, 1);   // the MMA thread's commit
-        }
-        for (int q = 0; q < SF; ++q) {
-            mbar_init(sf_full0 + 8 * q, 1);   // the scale issuer of the leader
-            mbar_init(sf_free0 + 8 * q, 1);   // the scale copier's commit
+            mbar_init(empty0 + 8 * s, 1);   // the MMA issuer's commit
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * Cfg::kEpiWarps);
@@ -234,58 +221,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         pn = tile - pm * num_pn;
     };
 
-    int issued = 0, sf_issued = 0;   // producers: code / scale stages whose loads this lane issued
-    int mma_done = 0;                // MMA thread: stages whose MMAs were issued
-    int copied = 0;                  // copier: stages whose scales were copied
-    if (warp == 0 && lane < 2 * S) {
-        // -------------------------------------------------------------- code producers (both CTAs)
-        const int op = lane / S, slot = lane % S;
-        if (lane == 0) {
+    int issued = 0;     // producer: stages whose loads were issued
+    int mma_done = 0;   // MMA warp: stages whose MMAs were issued
+    int copied = 0;     // copier warp: stages whose scales were copied
+    if (warp == 0) {
+        // -------------------------------------------------------------- producer (both CTAs)
+        if (elect_one()) {
             prefetch_tmap(&tmA);
             prefetch_tmap(&tmB);
-        }
-        const uint32_t full_leader0 = mapa_shared(full0, 0);
-        for (int it = slot; it < total; it += S) {
-            if (it >= S && !mbar_wait(empty0 + 8 * slot, ((it / S) & 1) ^ 1)) break;
-            int pm, pn, ks;
-            stage_tile(it, pm, pn, ks);
-            const uint32_t dst = smem_u32(base + slot * Cfg::kStageBytes + (op ? Cfg::kA : 0));
-            if (leader) mbar_arrive_expect_tx(full0 + 8 * slot, 2 * (op ? Cfg::kB : Cfg::kA));
-            if (op == 0)
-                tma_load_2d_pair(dst, &tmA, ks * 128, pm * 256 + (int)rank * 128, full_leader0 + 8 * slot);
-            else
-                tma_load_2d_pair(dst, &tmB, ks * 128, pn * 256 + (int)rank * 128, full_leader0 + 8 * slot);
-            issued = it + 1;
-        }
-    } else if (warp == 3 && lane < SF) {
-        // -------------------------------------------------------------- scale producers (both CTAs)
-        const int q = lane;
-        if (q == 0) {
             prefetch_tmap(&tmSFA);
             prefetch_tmap(&tmSFB);
         }
-        const uint32_t sf_full_leader0 = mapa_shared(sf_full0, 0);
-        for (int j = q; j < total; j += SF) {
-            if (j >= SF && !mbar_wait(sf_free0 + 8 * q, ((j / SF) & 1) ^ 1)) break;
+        __syncwarp();
+        const uint32_t full_leader0 = mapa_shared(full0, 0);
+        for (int it = 0; it < total; ++it) {
+            const int s = it % S;
+            if (it >= S && !mbar_wait_warp(empty0 + 8 * s, ((it / S) & 1) ^ 1)) break;
             int pm, pn, ks;
-            stage_tile(j, pm, pn, ks);
-            const uint32_t dst = smem_u32(sf_base + q * Cfg::kSfStageBytes);
-            if (leader) mbar_arrive_expect_tx(sf_full0 + 8 * q, 2 * (Cfg::kSfa + Cfg::kSfb));
-            tma_load_2d_pair(dst, &tmSFA, ks * 256, pm * 2 + (int)rank, sf_full_leader0 + 8 * q);
-            tma_load_2d_pair(dst + Cfg::kSfa, &tmSFB, ks * 256, pn * 2, sf_full_leader0 + 8 * q);
-            sf_issued = j + 1;
+            stage_tile(it, pm, pn, ks);
+            const uint32_t st = smem_u32(base + s * Cfg::kStageBytes);
+            const uint32_t fb = full_leader0 + 8 * s;
+            if (elect_one()) {
+                if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * Cfg::kStageBytes);
+                tma_load_2d_pair(st, &tmA, ks * 128, pm * 256 + (int)rank * 128, fb);
+                tma_load_2d_pair(st + Cfg::kA, &tmB, ks * 128, pn * 256 + (int)rank * 128, fb);
+                tma_load_2d_pair(st + Cfg::kA + Cfg::kB, &tmSFA, ks * 256, pm * 2 + (int)rank, fb);
+                tma_load_2d_pair(st + Cfg::kA + Cfg::kB + Cfg::kSfa, &tmSFB, ks * 256, pn * 2, fb);
+            }
+            __syncwarp();
+            issued = it + 1;
         }
-    } else if (warp == 1 && lane == 0 && leader) {
+    } else if (warp == 1 && leader) {
         // -------------------------------------------------------------- MMA issuer (leader)
         int it = 0;
         bool ok = true;
         for (int t_iter = 0; t_iter < my_tiles && ok; ++t_iter) {
-            if (t_iter > 0 && !mbar_wait(acc_empty, (t_iter - 1) & 1)) break;
+            if (t_iter > 0 && !mbar_wait_warp(acc_empty, (t_iter - 1) & 1)) break;
             tc_fence_after();
             for (int ks = 0; ks < nks; ++ks, ++it) {
                 const int s = it % S;
                 const uint32_t par = (it / S) & 1;
-                if (!mbar_wait(full0 + 8 * s, par) || !mbar_wait(sftm0 + 8 * s, par)) {
+                if (!mbar_wait_warp(full0 + 8 * s, par)) {
+                    ok = false;
+                    break;
+                }
+                if (!mbar_wait_warp(sftm0 + 8 * s, par)) {
                     ok = false;
                     break;
                 }
@@ -293,38 +273,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                 const int nk = min(4, nkb - ks * 4);
                 const uint32_t st = smem_u32(base + s * Cfg::kStageBytes);
                 const uint32_t t_sf = tmem + 256 + Cfg::kSfRegionCols * s;
-                for (int kk = 0; kk < nk; ++kk) {
-                    const uint64_t adesc = make_smem_desc(st + 32 * kk, 16, 1024, 2);
-                    const uint64_t bdesc = make_smem_desc(st + Cfg::kA + 32 * kk, 16, 1024, 2);
-                    tc_mma_pair_nvfp4(tmem, adesc, bdesc, Cfg::kIdesc, t_sf + 4 * kk, t_sf + 16 + 8 * kk,
-                                      (ks | kk) != 0);
+                if (elect_one()) {
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const uint64_t adesc = make_smem_desc(st + 32 * kk, 16, 1024, 2);
+                        const uint64_t bdesc = make_smem_desc(st + Cfg::kA + 32 * kk, 16, 1024, 2);
+                        tc_mma_pair_nvfp4(tmem, adesc, bdesc, Cfg::kIdesc, t_sf + 4 * kk, t_sf + 16 + 8 * kk,
+                                          (ks | kk) != 0);
+                    }
+                    tc_commit_pair_both(empty0 + 8 * s);
                 }
-                tc_commit_pair_both(empty0 + 8 * s);
+                __syncwarp();
                 mma_done = it + 1;
-                *consumed_slot = it + 1;
             }
-            if (ok) tc_commit_pair_both(acc_full);
+            if (ok) {
+                if (elect_one()) tc_commit_pair_both(acc_full);
+                __syncwarp();
+            }
         }
-    } else if (warp == 2 && lane == 0 && leader) {
+    } else if (warp == 2 && leader) {
         // -------------------------------------------------------------- scale copier (leader)
-        // A k-block's A scales are one atom (TMEM columns +4kb), its B scales two atoms (the B
-        // rows n and n + 128 of the tile; columns +16+8kb and +20+8kb).
+        // The stage's data landed, so the MMAs that last used its scale region completed.
         for (int j = 0; j < total; ++j) {
-            const int q = j % SF, r = j % S;
-            if (!mbar_wait(sf_full0 + 8 * q, (j / SF) & 1)) break;
-            if (j >= S && !mbar_wait(empty0 + 8 * r, ((j / S) & 1) ^ 1)) break;   // region r is free
+            const int s = j % S;
+            if (!mbar_wait_warp(full0 + 8 * s, (j / S) & 1)) break;
             tc_fence_after();
             const int nk = min(4, nkb - (j % nks) * 4);
-            const uint32_t sfa = smem_u32(sf_base + q * Cfg::kSfStageBytes);
-            const uint32_t sfb = sfa + Cfg::kSfa;
-            const uint32_t t_sf = tmem + 256 + Cfg::kSfRegionCols * r;
-            for (int kk = 0; kk < nk; ++kk) {
-                tc_cp_pair_32x128b_warpx4(t_sf + 4 * kk, make_smem_desc(sfa + 512 * kk, 0, 128, 0));
-                tc_cp_pair_32x128b_warpx4(t_sf + 16 + 8 * kk, make_smem_desc(sfb + 512 * kk, 0, 128, 0));
-                tc_cp_pair_32x128b_warpx4(t_sf + 20 + 8 * kk, make_smem_desc(sfb + 2048 + 512 * kk, 0, 128, 0));
+            const uint32_t sfa = smem_u32(base + s * Cfg::kStageBytes + Cfg::kA + Cfg::kB), sfb = sfa + Cfg::kSfa;
+            const uint32_t t_sf = tmem + 256 + Cfg::kSfRegionCols * s;
+            if (elect_one()) {
+                for (int kk = 0; kk < nk; ++kk) {
+                    tc_cp_pair_32x128b_warpx4(t_sf + 4 * kk, make_smem_desc(sfa + 512 * kk, 0, 128, 0));
+                    tc_cp_pair_32x128b_warpx4(t_sf + 16 + 8 * kk, make_smem_desc(sfb + 512 * kk, 0, 128, 0));
+                    tc_cp_pair_32x128b_warpx4(t_sf + 20 + 8 * kk, make_smem_desc(sfb + 2048 + 512 * kk, 0, 128, 0));
+                }
+                tc_commit_pair_leader(sftm0 + 8 * s);
             }
-            tc_commit_pair_leader(sftm0 + 8 * r);
-            tc_commit_pair_both(sf_free0 + 8 * q);
+            __syncwarp();
             copied = j + 1;
         }
     } else if (warp >= Cfg::kEpiWarp0) {
@@ -373,29 +357,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             }
         }
     }
-    issued = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)issued);
-    sf_issued = (int)__reduce_max_sync(0xFFFFFFFFu, (unsigned)sf_issued);
-    __syncwarp();
+    // Every role ends converged.  Only after a timeout can work still be in flight: the leader
+    // waits (bounded) for the loads it issued past the last consumed stage and for the last
+    // issued MMAs and copies, then both CTAs meet before TMEM is freed.
+    __shared__ int consumed, issued_here;
+    if (warp == 1 && leader && lane == 0) consumed = mma_done;
+    if (warp == 0 && lane == 0) issued_here = issued;
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();   // both CTAs are done issuing; the leader's counts are final
-    if (leader && threadIdx.x == 0) {
-        // Only after a timeout can work still be in flight: wait (bounded) for every issued
-        // stage's code loads ...
-        for (int it = *consumed_slot; it < issued; ++it) mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
-    }
-    if (leader && warp == 3 && lane == 0) {
-        // ... and scale loads (the newest one of each slot; older ones were copied)
-        for (int j = sf_issued > SF ? sf_issued - SF : 0; j < sf_issued; ++j)
-            mbar_wait(sf_full0 + 8 * (j % SF), (j / SF) & 1);
-    }
-    if (leader && warp == 2 && lane == 0 && copied > 0) {
-        const int j = copied - 1;
-        mbar_wait(sf_free0 + 8 * (j % SF), (j / SF) & 1);
+    cluster_sync_all();
+    if (leader && warp == 0 && lane == 0) {
+        // both SMs' loads of a stage complete on the leader's barrier
+        const int peer = (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&issued_here), 1));
+        const int last = max(issued, peer);
+        for (int it = consumed; it < last; ++it) mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
     }
     if (leader && warp == 1 && lane == 0 && mma_done > 0) {
         const int it = mma_done - 1;
         mbar_wait(empty0 + 8 * (it % S), (it / S) & 1);
+    }
+    if (leader && warp == 2 && lane == 0 && copied > 0) {
+        const int j = copied - 1;
+        mbar_wait(sftm0 + 8 * (j % S), (j / S) & 1);
     }
     cluster_sync_all();   // no SM frees TMEM or exits while its pair may still touch it
     tc_fence_after();
