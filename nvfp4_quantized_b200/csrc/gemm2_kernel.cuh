@@ -36,7 +36,7 @@
 //   warps 4..11        : epilogue.  Warp w reads TMEM lane quadrant w%4, columns [0, 128) for
 //                        warps 4..7 and [128, 256) for warps 8..11, all into registers, releases
 //                        the accumulator, then scales and stores its rows straight to global
-//                        memory (bf16 or fp32) while the next tile's MMAs run.
+//                        memory (bf16 or fp32, 32-byte stores) while the next tile's MMAs run.
 // Tensor memory: accumulator columns [0, 256); scale region s (of ring slot s) at 256 + 48 s
 // (A: 4 k-blocks x 4 columns, B: 4 k-blocks x 8 columns).
 // Every wait is bounded; on a timeout the CTA records QT2_ERR_TIMEOUT, the leader drains the
@@ -140,6 +140,13 @@ __device__ __forceinline__ void tc_commit_pair_leader(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
                      bar),
                  "h"(leader_only)
+                 : "memory");
+}
+
+// 32-byte global store (sm_100 256-bit vector store); the address is 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&p)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(p[0]), "r"(p[1]), "r"(p[2]),
+                 "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7])
                  : "memory");
 }
 
@@ -317,6 +324,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         const int cb = (ew >> 2) * 128;   // this warp's 128 of the tile's 256 columns
         const uint32_t acc_empty_leader = mapa_shared(acc_empty, 0);
         const float sc = alpha * (*gA) * (*gB);
+        const int64_t row_bytes = ldc * (c_dtype == QT2_DTYPE_F32 ? 4 : 2);
+        const bool wide = (reinterpret_cast<uintptr_t>(Cout) & 31) == 0 && (row_bytes & 31) == 0;
         for (int t_iter = 0; t_iter < my_tiles; ++t_iter) {
             if (!mbar_wait_warp(acc_full, t_iter & 1)) break;
             tc_fence_after();
@@ -335,24 +344,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            // 32-byte stores (each fills whole 32-byte sectors of its row) when C's rows are
+            // 32-byte aligned, else 16-byte stores
             if (c_dtype == QT2_DTYPE_F32) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + row * ldc + col);
+                float *dst = static_cast<float *>(Cout) + row * ldc + col;
+                if (wide) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    dst[i] = make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
-                                         __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc);
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t p[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) p[k] = __float_as_uint(__uint_as_float(v[8 * i + k]) * sc);
+                        st_global_v8(dst + 8 * i, p);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        reinterpret_cast<float4 *>(dst)[i] =
+                            make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
+                                        __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc);
+                }
             } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(Cout) + row * ldc + col);
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(Cout) + row * ldc + col;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    uint32_t p[4];
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t p[8];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2 * k]) * sc,
-                                                                  __uint_as_float(v[8 * i + 2 * k + 1]) * sc);
+                    for (int k = 0; k < 8; ++k) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[16 * i + 2 * k]) * sc,
+                                                                  __uint_as_float(v[16 * i + 2 * k + 1]) * sc);
                         p[k] = *reinterpret_cast<uint32_t *>(&b2);
                     }
-                    dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+                    if (wide) {
+                        st_global_v8(dst + 16 * i, p);
+                    } else {
+                        reinterpret_cast<uint4 *>(dst + 16 * i)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+                        reinterpret_cast<uint4 *>(dst + 16 * i)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+                    }
                 }
             }
         }

@@ -83,3 +83,27 @@ def test_gemm_zero_and_extreme_scales():
     got = gpu_gemm(va, vb, 1.0, qt2.QT2_DTYPE_F32)
     assert np.all(got[:128] == 0.0)
     check(got, va, vb, 1.0)
+
+
+# Output with a leading dimension larger than N, and a base 16 bytes off a 32-byte boundary: the
+# pair kernel stores 32 bytes at a time only when every row start is 32-byte aligned, else 16.
+# (dtype, extra columns, start offset in elements)
+PADDED = [(qt2.QT2_DTYPE_BF16, 8, 0), (qt2.QT2_DTYPE_BF16, 16, 0), (qt2.QT2_DTYPE_F32, 8, 4),
+          (qt2.QT2_DTYPE_F32, 8, 0)]
+
+
+@pytest.mark.parametrize("dtype,pad,off", PADDED)
+def test_gemm_strided_output(dtype, pad, off):
+    M, N, K = 512, 768, 1024
+    va = O.fwd46(_x(M, K, 8))
+    vb = O.fwd46(_x(N, K, 9, 0.02))
+    tdt = torch.float32 if dtype == qt2.QT2_DTYPE_F32 else torch.bfloat16
+    ldc = N + pad
+    buf = torch.full((off + M * ldc + 64,), 7.0, dtype=tdt, device="cuda")
+    out = buf[off:off + M * ldc].view(M, ldc)
+    qt2.qt2_gemm_nvfp4(upload(va), upload(vb), M, N, K, 1.0, out, dtype, ldc)
+    assert qt2.qt2_device_status() == 0
+    got = out[:, :N].float().cpu().numpy().astype(np.float64)
+    check(got, va, vb, 1.0, bf16=dtype == qt2.QT2_DTYPE_BF16)
+    assert torch.all(out[:, N:] == 7.0)          # padding columns untouched
+    assert torch.all(buf[:off] == 7.0) and torch.all(buf[off + M * ldc:] == 7.0)
