@@ -35,11 +35,15 @@ if ROOT not in sys.path:
 METRIC = "Quartet II linear fwd+bwd TFLOPS; quantizer GB/s; % of FP4/HBM roofline"
 UNIT = "TFLOP/s"
 KERNELS_PER_STEP = 13   # per step: 2 max + 2 fwd46 + 3 GEMM + 3 MS-EDEN producers + 3 finalize (dY views share one)
+# --schedule fused: X max + X's two views in one pass + its finalize, W max + fwd46, dY MS-EDEN +
+# finalize, 3 GEMMs (W's column view is made once, before the timed steps)
+KERNELS_PER_STEP_FUSED = 10
 
 # Algorithmic bytes per input element of each quantizer call (reads + writes the method needs).
 BYTES_FWD46 = 2 + 2 + 0.5 + 1 / 16            # max pass read, quantize read, codes, scales
 BYTES_MSED_ONE = 2 + 0.5 + 0.25 + 0.25 + 1 / 16  # read, codes, pre-scale write + read, scales
 BYTES_MSED_BOTH = 2 + 2 * (0.5 + 0.25 + 0.25 + 1 / 16)
+BYTES_FUSED_X = 2 + 2 + (0.5 + 1 / 16) + (0.5 + 0.25 + 0.25 + 1 / 16)   # max read, read, both views
 
 
 def peaks():
@@ -156,10 +160,39 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ws_w = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(N, K, COL), dev)
     ws_x = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(M, K, COL), dev)
     stream = torch.cuda.current_stream(dev)
-    names = ["fwd46_x", "fwd46_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col", "gemm_dgrad",
-             "gemm_wgrad"]
+    fused = args.schedule == "fused"
+    names = run_names(args.schedule)
+    seed0 = 0x5EED0000
+    if fused:
+        ws_xv = Q.alloc_workspace(Q.qt2_quant_fwd46_msedEN_col_workspace_size(M, K), dev)
+        # W's column view, made once for every micro-batch of the optimizer step (same seed)
+        Q.qt2_quant_msedEN(sets[0][1], N, K, K, COL, seed0, 0, Q.QT2_TID_W_COL, None, v_w_col, ws_w, ws_w.numel(),
+                           stream)
+
+    def step_fused(i, ev=None):
+        x, w, dy = sets[i % 2]
+
+        def mark(j):
+            if ev is not None:
+                ev[j].record(stream)
+        mark(0)
+        Q.qt2_quant_fwd46_msedEN_col(x, M, K, K, seed0, Q.QT2_TID_X_COL, vx, v_x_col, ws_xv, ws_xv.numel(), stream)
+        mark(1)
+        Q.qt2_quant_fwd46(w, N, K, K, ROW, vw, None, ws46b, ws46b.numel(), stream)
+        mark(2)
+        Q.qt2_gemm_nvfp4(vx, vw, M, N, K, 1.0, y, Q.QT2_DTYPE_BF16, N, stream)
+        mark(3)
+        Q.qt2_quant_msedEN(dy, M, N, N, BOTH, seed0, Q.QT2_TID_DY_ROW, Q.QT2_TID_DY_COL, v_dy_row, v_dy_col, ws_dy,
+                           ws_dy.numel(), stream)
+        mark(4)
+        Q.qt2_gemm_nvfp4(v_dy_row, v_w_col, M, K, N, 2.0 ** -7, dx, Q.QT2_DTYPE_BF16, K, stream)
+        mark(5)
+        Q.qt2_gemm_nvfp4(v_dy_col, v_x_col, N, K, M, 2.0 ** -7, dw, Q.QT2_DTYPE_F32, K, stream)
+        mark(6)
 
     def step(i, ev=None):
+        if fused:
+            return step_fused(i, ev)
         x, w, dy = sets[i % 2]
         seed = 0x5EED0000 + i
 
@@ -195,7 +228,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     assert Q.qt2_device_status(stream) == 0, "device status word set during warm-up"
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     clk.begin()
@@ -330,6 +363,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
+    ap.add_argument("--schedule", choices=["separate", "fused"], default="separate",
+                    help="fused: X's forward and column views from one read (qt2_quant_fwd46_msedEN_col) and "
+                         "W's column view made once and reused by every step, as micro-batches of one "
+                         "optimizer step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -398,23 +435,18 @@ def main():
     def gbs(bytes_, ms):
         return bytes_ / (ms * 1e-3) / 1e9
 
-    kernels = {
-        "gemm_fwd": {"ms": per["gemm_fwd"], "tflops": flops_gemm / (per["gemm_fwd"] * 1e-3) / 1e12},
-        "gemm_dgrad": {"ms": per["gemm_dgrad"], "tflops": flops_gemm / (per["gemm_dgrad"] * 1e-3) / 1e12},
-        "gemm_wgrad": {"ms": per["gemm_wgrad"], "tflops": flops_gemm / (per["gemm_wgrad"] * 1e-3) / 1e12},
-        "fwd46_x": {"ms": per["fwd46_x"], "gbs": gbs(M * K * BYTES_FWD46, per["fwd46_x"])},
-        "fwd46_w": {"ms": per["fwd46_w"], "gbs": gbs(N * K * BYTES_FWD46, per["fwd46_w"])},
-        "msed_dy_both": {"ms": per["msed_dy_both"], "gbs": gbs(M * N * BYTES_MSED_BOTH, per["msed_dy_both"])},
-        "msed_w_col": {"ms": per["msed_w_col"], "gbs": gbs(N * K * BYTES_MSED_ONE, per["msed_w_col"])},
-        "msed_x_col": {"ms": per["msed_x_col"], "gbs": gbs(M * K * BYTES_MSED_ONE, per["msed_x_col"])},
-    }
-    for k, v in kernels.items():
-        if "gbs" in v:
-            v["hbm_frac"] = v["gbs"] / pk["hbm_gbs"]
+    qbytes = quant_bytes_per_call(M, K, N)
+    kernels = {}
+    for n in per:
+        if n.startswith("gemm_"):
+            kernels[n] = {"ms": per[n], "tflops": flops_gemm / (per[n] * 1e-3) / 1e12}
+            kernels[n]["fp4_frac"] = kernels[n]["tflops"] / fp4_peak
         else:
-            v["fp4_frac"] = v["tflops"] / fp4_peak
-    quant_ms = sum(per[n] for n in names_quant())
-    quant_bytes = (M * K + N * K) * BYTES_FWD46 + M * N * BYTES_MSED_BOTH + (N * K + M * K) * BYTES_MSED_ONE
+            kernels[n] = {"ms": per[n], "gbs": gbs(qbytes[n], per[n])}
+            kernels[n]["hbm_frac"] = kernels[n]["gbs"] / pk["hbm_gbs"]
+    quant_names = [n for n in per if not n.startswith("gemm_")]
+    quant_ms = sum(per[n] for n in quant_names)
+    quant_bytes = sum(qbytes[n] for n in quant_names)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": r["max_ms"] / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -423,7 +455,7 @@ def main():
         "config": {"workload": workload, "M": M, "K": K, "N": N,
                    "parallelism": f"dp{world}: every rank its own token batch, no collective on the path",
                    "l2": "inputs larger than L2: two 352 MiB input sets alternate between steps",
-                   "output": "Y bf16, dX bf16, dW fp32"},
+                   "output": "Y bf16, dX bf16, dW fp32", "schedule": args.schedule},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp4_peak, "traffic": traffic,
                      "kernel": "gemm_nvfp4_pair_kernel (mean of the fwd, dgrad and wgrad launches)",
@@ -433,7 +465,7 @@ def main():
                        "hbm_frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                        "peak_gbs": pk["hbm_gbs"], "ms_per_step": quant_ms},
         "kernels": kernels,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP_FUSED if args.schedule == "fused" else KERNELS_PER_STEP) * args.steps,
         "clocks": r["clocks"],
         "device_status": r["status"],
     }
@@ -450,8 +482,18 @@ def main():
         dist.destroy_process_group()
 
 
-def names_quant():
-    return ["fwd46_x", "fwd46_w", "msed_dy_both", "msed_w_col", "msed_x_col"]
+def run_names(schedule: str):
+    """The calls of one step, in order (each is timed with CUDA events)."""
+    if schedule == "fused":
+        return ["fused_x_views", "fwd46_w", "gemm_fwd", "msed_dy_both", "gemm_dgrad", "gemm_wgrad"]
+    return ["fwd46_x", "fwd46_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col", "gemm_dgrad", "gemm_wgrad"]
+
+
+def quant_bytes_per_call(M: int, K: int, N: int):
+    """Algorithmic bytes of each quantizer call of a step."""
+    return {"fwd46_x": M * K * BYTES_FWD46, "fwd46_w": N * K * BYTES_FWD46, "msed_dy_both": M * N * BYTES_MSED_BOTH,
+            "msed_w_col": N * K * BYTES_MSED_ONE, "msed_x_col": M * K * BYTES_MSED_ONE,
+            "fused_x_views": M * K * BYTES_FUSED_X}
 
 
 if __name__ == "__main__":

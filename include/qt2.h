@@ -204,6 +204,40 @@ QT2_API qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, 
                           uint64_t seed, void *dx_bf16, void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
                           qt2_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Both views of a layer input from one read ([FAF] "the speed-up is lost between the
+ * matmuls": a producer that emits every layout the GEMMs need from one read of the tensor;
+ * the pages stress fusing the quantizers around the GEMMs).  x_bf16 [rows][cols] (ld):
+ *   row_out: the forward view (R = rows, C = cols), exactly what qt2_quant_fwd46 gives;
+ *   col_out: the MS-EDEN column view of x^T (R = cols, C = rows), exactly what
+ *            qt2_quant_msedEN gives with QT2_LAYOUT_COL, the same seed and tensor_id_col.
+ * A max pass over x comes first (the forward codes depend on the tensor scale), then one pass
+ * reads x once for both views.  For a layer, call it on X with the seed and QT2_TID_X_COL that
+ * the backward will use, and pass col_out to qt2_linear_bwd_views.
+ * Workspace: at least qt2_quant_fwd46_msedEN_col_workspace_size() bytes, 256-byte aligned.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_fwd46_msedEN_col_workspace_size(int64_t rows, int64_t cols, size_t *bytes);
+QT2_API qt2_status qt2_quant_fwd46_msedEN_col(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                              uint64_t seed, uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
+                                              const qt2_nvfp4_view *col_out, void *workspace, size_t ws_bytes,
+                                              qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Backward of the linear layer from column views quantized beforehand: x_col is X's MS-EDEN
+ * column view ([K][M] view, e.g. from qt2_quant_fwd46_msedEN_col), w_col is W's MS-EDEN column
+ * view ([K][N] view, qt2_quant_msedEN with QT2_LAYOUT_COL), both made with the same `seed` as
+ * this call (the rotation is shared) and tensor ids QT2_TID_X_COL / QT2_TID_W_COL to match
+ * qt2_linear_bwd.  W's view can be made once and reused by every micro-batch that runs with
+ * that seed.  dY gets both views here (QT2_TID_DY_ROW / _COL); then dX = dY W and dW = dY^T X
+ * as qt2_linear_bwd, whose results it reproduces bit for bit for the same inputs.
+ * Workspace: at least qt2_linear_bwd_views_workspace_size() bytes, 256-byte aligned.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_linear_bwd_views_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes);
+QT2_API qt2_status qt2_linear_bwd_views(const void *dy, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                                        const qt2_nvfp4_view *x_col, const qt2_nvfp4_view *w_col, void *dx_bf16,
+                                        void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
+                                        qt2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,10 @@
 //
 // The same producer serves the elementwise-SR baseline (qt2_quant_sr): kModeMax merges max |y|
 // of the rotated view(s) and writes nothing else; kModeSr then quantizes with that tensor scale
-// (sr_vector).  kModeEden is MS-EDEN.
+// (sr_vector).  kModeEden is MS-EDEN.  kModeFwdRowEdenCol gives both of X's views from one read
+// ([FAF]): the row warps quantize the tile's rows for the forward GEMM (RTN with the 4/6 choice,
+// as fwd46_rows_kernel, with the tensor max of X taken beforehand), the column warps produce the
+// MS-EDEN column view.
 #pragma once
 
 #include "quant_kernels.cuh"
@@ -291,7 +294,7 @@ struct RotViews {
     float *row_g, *col_g;               // SR tensor scales, written
     uint32_t tid_row, tid_col;          // SR Philox tensor ids
 };
-enum RotMode { kModeEden = 0, kModeMax = 1, kModeSr = 2 };
+enum RotMode { kModeEden = 0, kModeMax = 1, kModeSr = 2, kModeFwdRowEdenCol = 3 };
 
 template <int MODE, bool DO_ROW, bool DO_COL>
 __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
@@ -326,6 +329,15 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         mbar_arrive_expect_tx(fb, Cfg::kTileBytes);
         tma_load_2d(smem_u32(buf0 + s * Cfg::kTileBytes), &tmap, c0, r0, fb);
         tma_load_2d(smem_u32(buf0 + s * Cfg::kTileBytes + 16384), &tmap, c0 + 64, r0, fb);
+    };
+    // A warp is done reading stage s (tile i); the last of the tile's readers refills the stage.
+    auto release = [&](int s, int64_t i) {
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence_block();
+            const uint32_t old = atomicAdd(&done_cnt[s], 1u);
+            if (old == (uint32_t)(i / NS + 1) * kConsumers - 1 && i + NS < my_tiles) issue(i + NS);
+        }
     };
     if (t == 0) {
         prefetch_tmap(&tmap);
@@ -365,6 +377,17 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             if (blockIdx.x == 0 && t == 0) *out.col_g = g_c;
         }
     }
+    // forward view of the rows (kModeFwdRowEdenCol): tensor scale and the block's scale tables
+    __shared__ float tab_d[128], tab_r[128];
+    float g6_f = 0.0f, g4_f = 0.0f;
+    if constexpr (MODE == kModeFwdRowEdenCol) {
+        const float g = fwd46_tensor_scale(row_amax);
+        g6_f = __fmul_rn(g, 6.0f);
+        g4_f = __fmul_rn(g, 4.0f);
+        if (blockIdx.x == 0 && t == 0) *out.row_g = g;
+        fwd46_tables(g, tab_d, tab_r);
+        __syncthreads();
+    }
     const float sigma = h ? -1.0f : 1.0f;
     const uint64_t sg = f2(sigma, sigma), nsg = f2(-sigma, -sigma);
     const bool rows = kBoth ? team == 0 : DO_ROW;
@@ -381,6 +404,29 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         // A tile is two 128x64 boxes with the 128-byte swizzle: element (r, c) sits at byte
         // (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
         const uint32_t tbu = smem_u32(tb);
+        if constexpr (MODE == kModeFwdRowEdenCol) {
+            if (rows) {
+                // forward view of row u: groups 4h .. 4h+3 of the block (elements [64h, 64h + 64),
+                // chunks c ^ (u % 8) of box h), quantized straight from shared memory; codes at
+                // bytes [32h, 32h + 32) of the block, one scale word; then the stage is released
+                const uint32_t rbase = tbu + h * 16384 + u * 128;
+                uint32_t cw[8], scw = 0;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    const uint4 a = lds128(rbase + ((uint32_t)((2 * gq) ^ (u & 7)) << 4));
+                    const uint4 b = lds128(rbase + ((uint32_t)((2 * gq + 1) ^ (u & 7)) << 4));
+                    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    scw |= fwd46_group(w, g6_f, g4_f, tab_d, tab_r, cw[2 * gq], cw[2 * gq + 1]) << (8 * gq);
+                }
+                release(s, i);
+                const int64_t vr = r0 + u;
+                uint8_t *const vcodes = row_codes + vr * (C >> 1) + (c0 >> 1);
+                *reinterpret_cast<uint4 *>(vcodes + 32 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                *reinterpret_cast<uint4 *>(vcodes + 32 * h + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                *reinterpret_cast<uint32_t *>(out.row_scales + sf_offset(vr, (c0 >> 4) + 4 * h, C)) = scw;
+                continue;
+            }
+        }
         if (rows) {
             // row u, elements [64h, 64h + 64); register chunk c holds element chunk 8h + (c ^ 4h),
             // whose 16 bytes sit at swizzled chunk (c ^ 4h ^ (u % 8)) of row u in box h
@@ -428,12 +474,7 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             }
         }
         // The tile is in registers: release the stage; the last warp to do so refills it.
-        __syncwarp();
-        if (lane == 0) {
-            __threadfence_block();
-            const uint32_t old = atomicAdd(&done_cnt[s], 1u);
-            if (old == (uint32_t)(i / NS + 1) * kConsumers - 1 && i + NS < my_tiles) issue(i + NS);
-        }
+        release(s, i);
         const int64_t vr = rows ? r0 + u : c0 + u;   // view row (the column view is [C][R])
         const int64_t VC = rows ? C : R, b0 = rows ? c0 : r0;   // view row length, block start
         uint8_t *const vcodes = (rows ? row_codes : col_codes) + vr * (VC >> 1) + (b0 >> 1);
@@ -442,6 +483,11 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             float Pq[4];
             msed_vector(P, sg, nsg, cw, Pq, amax);
             msed_store(vcodes, rows ? row_P : col_P, vr, b0 >> 4, VC, h, cw, Pq);
+        } else if constexpr (MODE == kModeFwdRowEdenCol) {   // column warps (rows returned above)
+            uint32_t cw[8];
+            float Pq[4];
+            msed_vector(P, sg, nsg, cw, Pq, amax);
+            msed_store(vcodes, col_P, vr, b0 >> 4, VC, h, cw, Pq);
         } else if constexpr (MODE == kModeMax) {
             rotate_tail(P, sg, nsg);
 #pragma unroll
@@ -467,8 +513,9 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         }
     }
     if constexpr (MODE != kModeSr) {
+        // (kModeFwdRowEdenCol: the row warps merge nothing; row_amax is the input's max)
         const uint32_t bm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax));
-        if (lane == 0 && bm != 0) atomicMax(rows ? row_amax : col_amax, bm);
+        if (lane == 0 && bm != 0 && !(MODE == kModeFwdRowEdenCol && rows)) atomicMax(rows ? row_amax : col_amax, bm);
     }
     __syncthreads();
     if (t == 0) {

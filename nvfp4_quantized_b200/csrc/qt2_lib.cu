@@ -92,6 +92,21 @@ cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, boo
     return launch_rot<kModeEden>(tmap, R, C, do_row, do_col, seed, out, s);
 }
 
+// X's forward row view and MS-EDEN column view from one read (amax_x: the max pass's word,
+// read; amax_col: the column view's max |y|, merged).
+cudaError_t launch_fwd46_msed_col(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed, DevView row,
+                                  DevView col, float *P_col, uint32_t *amax_x, uint32_t *amax_col, cudaStream_t s) {
+    RotViews out{};
+    out.row_codes = row.codes;
+    out.row_scales = row.scales;
+    out.row_g = row.tensor_scale;
+    out.row_amax = amax_x;
+    out.col_codes = col.codes;
+    out.col_P = P_col;
+    out.col_amax = amax_col;
+    return launch_rot_variant<kModeFwdRowEdenCol, true, true>(tmap, R, C, seed, out, s);
+}
+
 static FinalizeJob finalize_job(const float *P, int64_t R, int64_t C, const uint32_t *amax_word, uint32_t tid,
                                 DevView out, int64_t max_blocks) {
     const int64_t words = (R * C) >> 6;
@@ -289,6 +304,25 @@ qt2_status msed_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, i
     return from_cuda(e);
 }
 
+// X's forward view and MS-EDEN column view: max pass, one fused pass, the column view's finalize.
+// amax: 2 words (the input's max |x|, the column view's max |y|).
+qt2_status fwd46_msed_col_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
+                                  uint32_t tid_col, DevView row, DevView col, float *P_col, uint32_t *amax,
+                                  cudaStream_t s) {
+    CUtensorMap tmap;
+    if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
+                        128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return QT2_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_fwd46_msed_col(tmap, rows, cols, seed, row, col, P_col, amax, amax + 1, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    return from_cuda(
+        launch_msed_finalize(P_col, cols, rows, amax + 1, tid_col, col, nullptr, 0, 0, nullptr, 0, col, seed, s));
+}
+
 qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *amax,
                          cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s);
@@ -359,6 +393,23 @@ size_t linear_bwd_layout(int64_t M, int64_t K, int64_t N, void *ws, BwdLayout *L
     L->P_dy_col = reinterpret_cast<float *>(c.take((size_t)M * N / 16 * 4));
     L->P_w_col = reinterpret_cast<float *>(c.take((size_t)N * K / 16 * 4));
     L->P_x_col = reinterpret_cast<float *>(c.take((size_t)M * K / 16 * 4));
+    return c.used;
+}
+
+// Workspace of qt2_linear_bwd_views: dY's two views and their pre-scales.
+struct BwdViewsLayout {
+    DevView dy_row, dy_col;
+    float *P_dy_row, *P_dy_col;
+    uint32_t *amax;   // 2 words: dY row, col
+};
+
+size_t linear_bwd_views_layout(int64_t M, int64_t N, void *ws, BwdViewsLayout *L) {
+    Carve c(ws);
+    L->amax = reinterpret_cast<uint32_t *>(c.take(2 * sizeof(uint32_t)));
+    L->dy_row = carve_view(c, M, N);
+    L->dy_col = carve_view(c, N, M);
+    L->P_dy_row = reinterpret_cast<float *>(c.take((size_t)M * N / 16 * 4));
+    L->P_dy_col = reinterpret_cast<float *>(c.take((size_t)M * N / 16 * 4));
     return c.used;
 }
 
@@ -627,6 +678,65 @@ qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t 
     if ((st = gemm_enqueue(L.dy_row, L.w_col, M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK) return st;
     // wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
     return gemm_enqueue(L.dy_col, L.x_col, N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
+}
+
+qt2_status qt2_quant_fwd46_msedEN_col_workspace_size(int64_t rows, int64_t cols, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols)) return QT2_ERR_SHAPE;
+    float *a, *b;
+    uint32_t *c;
+    *bytes = msed_ws(rows, cols, QT2_LAYOUT_COL, &a, &b, &c, nullptr);
+    return QT2_OK;
+}
+
+qt2_status qt2_quant_fwd46_msedEN_col(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, uint64_t seed,
+                                      uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
+                                      const qt2_nvfp4_view *col_out, void *workspace, size_t ws_bytes,
+                                      qt2_stream_t stream) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!view_ok(col_out)) return col_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    float *P_row, *P_col;
+    uint32_t *amax;
+    if (ws_bytes < msed_ws(rows, cols, QT2_LAYOUT_COL, &P_row, &P_col, &amax, workspace)) return QT2_ERR_WORKSPACE;
+    if ((st = check_device()) != QT2_OK) return st;
+    return fwd46_msed_col_enqueue(x_bf16, rows, cols, ld, seed, tensor_id_col, dev_view(row_out), dev_view(col_out),
+                                  P_col, amax, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qt2_status qt2_linear_bwd_views_workspace_size(int64_t M, int64_t K, int64_t N, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    BwdViewsLayout L;
+    *bytes = linear_bwd_views_layout(M, N, nullptr, &L);
+    return QT2_OK;
+}
+
+qt2_status qt2_linear_bwd_views(const void *dy, int64_t M, int64_t K, int64_t N, uint64_t seed,
+                                const qt2_nvfp4_view *x_col, const qt2_nvfp4_view *w_col, void *dx_bf16, void *dw,
+                                int dw_dtype, void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    if (!dy || !x_col || !w_col || !dx_bf16 || !dw) return QT2_ERR_INVALID_ARG;
+    if (dw_dtype != QT2_DTYPE_BF16 && dw_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
+    if (!view_ok(x_col) || !view_ok(w_col)) return QT2_ERR_ALIGN;
+    if (!aligned16(dy) || !aligned16(dx_bf16) || !aligned16(dw)) return QT2_ERR_ALIGN;
+    if (!workspace) return QT2_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsAlign - 1)) != 0) return QT2_ERR_ALIGN;
+    BwdViewsLayout L;
+    if (ws_bytes < linear_bwd_views_layout(M, N, workspace, &L)) return QT2_ERR_WORKSPACE;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = msed_enqueue(dy, M, N, N, QT2_LAYOUT_BOTH, seed, QT2_TID_DY_ROW, QT2_TID_DY_COL, L.dy_row, L.dy_col,
+                           L.P_dy_row, L.P_dy_col, L.amax, s)) != QT2_OK)
+        return st;
+    // dgrad: dX[M][K] = 2^-7 * dY_row[M][N] . W_col[K][N]^T; wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
+    if ((st = gemm_enqueue(L.dy_row, dev_view(w_col), M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK)
+        return st;
+    return gemm_enqueue(L.dy_col, dev_view(x_col), N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
 }
 
 }  // extern "C"

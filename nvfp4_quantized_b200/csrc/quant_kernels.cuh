@@ -149,21 +149,70 @@ __device__ __forceinline__ void fwd46_candidate(const uint64_t (&X)[8], const Fw
     }
 }
 
-__global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
-                                                         int64_t ld, const uint32_t *__restrict__ amax_word,
-                                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                                                         float *__restrict__ tensor_scale) {
-    const float A = __uint_as_float(*amax_word);
-    const bool zero_tensor = !(A >= kTiny);
-    const float g = zero_tensor ? 1.0f : __fdiv_rn(A, kFwd46Denominator);
-    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-    __shared__ float tab_d[128], tab_r[128];
+// The block's tables of d = RN(val(c) * g) and RN(1/d) for the 128 non-negative E4M3 codes c
+// (tab_r[0] = 0); called by the first 128 threads, followed by a barrier.
+__device__ __forceinline__ void fwd46_tables(float g, float *tab_d, float *tab_r) {
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(e4m3_value(threadIdx.x), g);
         tab_d[threadIdx.x] = d;
         tab_r[threadIdx.x] = threadIdx.x == 0 ? 0.0f : __frcp_rn(d);
     }
+}
+
+// One 16-element group (8 words of bf16 pairs, element 2i in the low half of word i): its two
+// code words and its scale code.
+__device__ __forceinline__ uint32_t fwd46_group(const uint32_t (&w)[8], float g6, float g4, const float *tab_d,
+                                                const float *tab_r, uint32_t &code0, uint32_t &code1) {
+    uint64_t X[8];
+    float m8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+        X[i] = f2(lo, hi);
+        m8[i] = fmaxf(fabsf(lo), fabsf(hi));
+    }
+#pragma unroll
+    for (int s = 8; s > 1; s >>= 1) {
+#pragma unroll
+        for (int i = 0; i < s / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
+    }
+    const float a = m8[0];
+    const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
+    uint32_t c6[2], c4[2];
+    float e6[8], e4[8];
+    fwd46_candidate(X, s6, c6, e6);
+    fwd46_candidate(X, s4, c4, e4);
+    uint64_t t[8];   // (candidate 6, candidate 4) level-1 sums, then levels 2..4 together
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
+#pragma unroll
+    for (int s = 8; s > 1; s >>= 1) {
+#pragma unroll
+        for (int i = 0; i < s / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
+    }
+    float err6, err4;
+    f2_split(t[0], err6, err4);
+    const bool pick4 = err4 < err6;                    // a tie keeps the full grid
+    code0 = pick4 ? c4[0] : c6[0];
+    code1 = pick4 ? c4[1] : c6[1];
+    return pick4 ? s4.code : s6.code;
+}
+
+// g = A/1792 of a tensor whose max |x| is A (1 for a zero tensor).
+__device__ __forceinline__ float fwd46_tensor_scale(const uint32_t *amax_word) {
+    const float A = __uint_as_float(*amax_word);
+    return (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
+}
+
+__global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
+                                                         int64_t ld, const uint32_t *__restrict__ amax_word,
+                                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                         float *__restrict__ tensor_scale) {
+    const float g = fwd46_tensor_scale(amax_word);
+    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
+    __shared__ float tab_d[128], tab_r[128];
+    fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
 
     const uint32_t G = (uint32_t)(C >> 4);                 // groups per row (a multiple of 8)
@@ -177,39 +226,8 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
         const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (uint64_t)q * 16);
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint64_t X[8];
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-            X[i] = f2(lo, hi);
-            m8[i] = fmaxf(fabsf(lo), fabsf(hi));
-        }
-#pragma unroll
-        for (int s = 8; s > 1; s >>= 1) {
-#pragma unroll
-            for (int i = 0; i < s / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
-        }
-        const float a = m8[0];
-        const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
-        uint32_t c6[2], c4[2];
-        float e6[8], e4[8];
-        fwd46_candidate(X, s6, c6, e6);
-        fwd46_candidate(X, s4, c4, e4);
-        uint64_t t[8];   // (candidate 6, candidate 4) level-1 sums, then levels 2..4 together
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
-#pragma unroll
-        for (int s = 8; s > 1; s >>= 1) {
-#pragma unroll
-            for (int i = 0; i < s / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
-        }
-        float err6, err4;
-        f2_split(t[0], err6, err4);
-        const bool pick4 = err4 < err6;                    // a tie keeps the full grid
-        const uint32_t code0 = pick4 ? c4[0] : c6[0];
-        const uint32_t code1 = pick4 ? c4[1] : c6[1];
-        const uint32_t sc = pick4 ? s4.code : s6.code;
+        uint32_t code0, code1;
+        const uint32_t sc = fwd46_group(w, g6, g4, tab_d, tab_r, code0, code1);
         *reinterpret_cast<uint2 *>(codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8) = make_uint2(code0, code1);
         // four consecutive groups (same row, q % 4 == 0 .. 3) share one scale word
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);

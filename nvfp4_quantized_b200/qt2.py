@@ -70,6 +70,10 @@ def lib() -> ctypes.CDLL:
                 "qt2_linear_fwd": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
                 "qt2_linear_bwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_bwd": (i32, [vp, vp, vp, i64, i64, i64, u64, vp, vp, i32, vp, sz, vp]),
+                "qt2_quant_fwd46_msedEN_col_workspace_size": (i32, [i64, i64, psz]),
+                "qt2_quant_fwd46_msedEN_col": (i32, [vp, i64, i64, i64, u64, u32, pv, pv, vp, sz, vp]),
+                "qt2_linear_bwd_views_workspace_size": (i32, [i64, i64, i64, psz]),
+                "qt2_linear_bwd_views": (i32, [vp, i64, i64, i64, u64, pv, pv, vp, vp, i32, vp, sz, vp]),
             }
             for name, (res, args) in sigs.items():
                 fn = getattr(L, name)
@@ -249,3 +253,34 @@ def qt2_linear_bwd(dy: torch.Tensor, x: torch.Tensor, w: torch.Tensor, M: int, K
                    stream=None) -> None:
     _check("qt2_linear_bwd", lib().qt2_linear_bwd(_ptr(dy), _ptr(x), _ptr(w), M, K, N, seed, _ptr(dx), _ptr(dw),
                                                   dw_dtype, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def qt2_quant_fwd46_msedEN_col_workspace_size(rows: int, cols: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qt2_quant_fwd46_msedEN_col_workspace_size",
+           lib().qt2_quant_fwd46_msedEN_col_workspace_size(rows, cols, ctypes.byref(n)))
+    return n.value
+
+
+def qt2_quant_fwd46_msedEN_col(x: torch.Tensor, rows: int, cols: int, ld: int, seed: int, tensor_id_col: int,
+                               row_out: View, col_out: View, workspace: torch.Tensor, ws_bytes: int,
+                               stream=None) -> None:
+    r, c = row_out.c(), col_out.c()
+    _check("qt2_quant_fwd46_msedEN_col", lib().qt2_quant_fwd46_msedEN_col(
+        _ptr(x), rows, cols, ld, seed, tensor_id_col, ctypes.byref(r), ctypes.byref(c), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
+def qt2_linear_bwd_views_workspace_size(M: int, K: int, N: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qt2_linear_bwd_views_workspace_size", lib().qt2_linear_bwd_views_workspace_size(M, K, N, ctypes.byref(n)))
+    return n.value
+
+
+def qt2_linear_bwd_views(dy: torch.Tensor, M: int, K: int, N: int, seed: int, x_col: View, w_col: View,
+                         dx: torch.Tensor, dw: torch.Tensor, dw_dtype: int, workspace: torch.Tensor, ws_bytes: int,
+                         stream=None) -> None:
+    xc, wc = x_col.c(), w_col.c()
+    _check("qt2_linear_bwd_views", lib().qt2_linear_bwd_views(
+        _ptr(dy), M, K, N, seed, ctypes.byref(xc), ctypes.byref(wc), _ptr(dx), _ptr(dw), dw_dtype, _ptr(workspace),
+        ws_bytes, _stream(stream)))

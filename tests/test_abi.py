@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 15
+    assert len(names) == 19
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -88,6 +88,22 @@ def test_host_validation_codes(L):
     assert L.qt2_linear_fwd(0x1000, 0x2000, 128, 128, 128, 0x3000, None, 0, None) == qt2.QT2_ERR_WORKSPACE
     assert L.qt2_linear_bwd(0x1000, 0x2000, 0x3000, 128, 128, 128, 0, 0x4000, 0x5000, 3, 0x6000, 1 << 30,
                             None) == qt2.QT2_ERR_INVALID_ARG
+    fx = L.qt2_quant_fwd46_msedEN_col
+    assert fx(0x1000, 128, 128, 128, 1, 4, R(v), None, 0x40000, 1 << 20, None) == qt2.QT2_ERR_INVALID_ARG
+    assert fx(0x1000, 128, 192, 192, 1, 4, R(v), R(v), 0x40000, 1 << 20, None) == qt2.QT2_ERR_SHAPE
+    assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(v), 0x40000, 16, None) == qt2.QT2_ERR_WORKSPACE
+    assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(_view(scales=0x20004)), 0x40000, 1 << 20,
+              None) == qt2.QT2_ERR_ALIGN
+    bv = L.qt2_linear_bwd_views
+    assert bv(0x1000, 128, 128, 128, 0, None, R(v), 0x4000, 0x5000, 1, 0x6000, 1 << 30, None) == \
+        qt2.QT2_ERR_INVALID_ARG
+    assert bv(0x1000, 128, 128, 128, 0, R(v), R(v), 0x4000, 0x5000, 9, 0x6000, 1 << 30, None) == \
+        qt2.QT2_ERR_INVALID_ARG
+    assert bv(0x1000, 128, 320, 128, 0, R(v), R(v), 0x4000, 0x5000, 1, 0x6000, 1 << 30, None) == qt2.QT2_ERR_SHAPE
+    assert bv(0x1000, 128, 128, 128, 0, R(v), R(v), 0x4000, 0x5000, 1, 0x6000, 64, None) == qt2.QT2_ERR_WORKSPACE
+    assert qt2.qt2_linear_bwd_views_workspace_size(256, 128, 384) < qt2.qt2_linear_bwd_workspace_size(256, 128, 384)
+    assert qt2.qt2_quant_fwd46_msedEN_col_workspace_size(256, 512) == \
+        qt2.qt2_quant_msedEN_workspace_size(256, 512, qt2.QT2_LAYOUT_COL)
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
