@@ -66,6 +66,7 @@ def lib():
                 "or_amax_bf16": (f32, [vp, i64]),
                 "or_fwd46_tensor_scale": (f32, [f32]),
                 "or_fwd46_rows": (None, [vp, i64, i64, f32, i64, i64, vp, vp, vp, vp, vp]),
+                "or_fwd46_sq_blocks": (None, [vp, i64, i64, f32, i64, i64, vp, vp, vp, vp, vp]),
                 "or_msedEN_rows_stage1": (None, [vp, i64, i64, vp, i64, i64, vp, vp, vp, vp]),
                 "or_msedEN_tensor_scale": (f32, [f32]),
                 "or_msedEN_finalize": (None, [vp, i64, i64, f32, u64, u32, i64, i64, vp]),
@@ -225,6 +226,40 @@ def fwd46(x, A: float | None = None) -> View:
                                              _p(e6), _p(e4)), R)
     return View(codes, scales, lib().or_fwd46_tensor_scale(A), amax=np.float32(A), choice=choice,
                 err6=e6, err4=e4)
+
+
+def transpose_codes(codes: np.ndarray) -> np.ndarray:
+    """Packed E2M1 codes of the transposed matrix: [R][C/2] -> [C][R/2] (data movement only)."""
+    R, C2 = codes.shape
+    nib = np.empty((R, 2 * C2), np.uint8)
+    nib[:, 0::2] = codes & 0xF
+    nib[:, 1::2] = codes >> 4
+    t = np.ascontiguousarray(nib.T)
+    return (t[:, 0::2] | (t[:, 1::2] << 4)).astype(np.uint8)
+
+
+def fwd46_sq(x, A: float | None = None) -> tuple[View, View]:
+    """Square-block forward quantizer of a bf16 [R][C] matrix: one scale per 16x16 block, the
+    forward quantizer's RTN and 4/6 choice per block (see or_fwd46_sq_blocks).  Returns the row
+    view ([R][C], groups along C) and the column view ([C][R], groups along R): the same
+    quantized values, transposed -- the one quantization serves both views of a weight."""
+    b = _bf16_bits(x)
+    R, C = b.shape
+    if A is None:
+        A = amax_bf16(b)
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    choice = np.zeros((R // 16, C // 16), np.uint8)
+    e6 = np.zeros((R // 16, C // 16), np.float32)
+    e4 = np.zeros((R // 16, C // 16), np.float32)
+    _rows(lambda b0, b1: lib().or_fwd46_sq_blocks(_p(b), R, C, A, b0, b1, _p(codes), _p(scales), _p(choice),
+                                                  _p(e6), _p(e4)), R // 16)
+    g = lib().or_fwd46_tensor_scale(A)
+    blk = scales[0::16]                                   # [R/16][C/16]: the block scales
+    col_scales = np.ascontiguousarray(np.repeat(blk.T, 16, axis=0))   # [C][R/16]
+    row = View(codes, scales, g, amax=np.float32(A), choice=choice, err6=e6, err4=e4)
+    col = View(transpose_codes(codes), col_scales, g, amax=np.float32(A))
+    return row, col
 
 
 def msedEN(x, seed: int, tid: int, view: str = "row") -> View:

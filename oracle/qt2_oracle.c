@@ -292,6 +292,63 @@ OR_EXPORT void or_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, float A, i
     }
 }
 
+/* Square-block forward quantizer over block rows [b0, b1) of a bf16 [R][C] matrix (R, C
+ * multiples of 16): one E4M3 scale per 16x16 block, so that the quantized matrix and its
+ * transpose are the same quantization and one pass serves both operand views of a weight
+ * ([QII-tg] "Method": the pages compare 16x16 blocks with 1x16 groups and keep the groups for
+ * their lower error; the square blocks are their faster alternative).  The steps are the forward
+ * quantizer's ones with the block in place of the group: a = max|x| over the block, for k = 6
+ * and k = 4 the scale E4M3_RNE(a/(g*k)) and the RTN codes of each of the 16 rows, the block's
+ * squared error = balanced tree over its 256 elements in row-major order (= the tree of the 16
+ * rows' 16-element trees); keep 4 iff its error is smaller (a tie keeps 6).
+ * Outputs in the row view's canonical layouts: codes [R][C/2], scales [R][C/16] (every row of a
+ * block repeats the block's scale); per block (nullable): choice, err6, err4 [R/16][C/16]. */
+OR_EXPORT void or_fwd46_sq_blocks(const uint16_t *x, int64_t R, int64_t C, float A, int64_t b0, int64_t b1,
+                                  uint8_t *codes, uint8_t *scales, uint8_t *choice, float *err6, float *err4)
+{
+    (void)R;
+    float g = or_fwd46_tensor_scale(A);
+    int zero_tensor = !(A >= OR_TINY);
+    int64_t G = C / 16;
+    for (int64_t rb = b0; rb < b1; rb++) {
+        for (int64_t q = 0; q < G; q++) {
+            float xv[16][16], a = 0.0f;
+            for (int i = 0; i < 16; i++)
+                for (int j = 0; j < 16; j++) {
+                    xv[i][j] = or_bf16_to_f32(x[(rb * 16 + i) * C + q * 16 + j]);
+                    if (fabsf(xv[i][j]) > a) a = fabsf(xv[i][j]);
+                }
+            uint8_t c6[16][16], c4[16][16], s6 = 0, s4 = 0;
+            float r6[16], r4[16];
+            for (int i = 0; i < 16; i++) {
+                if (zero_tensor) {
+                    float sq[16];
+                    for (int j = 0; j < 16; j++) {
+                        c6[i][j] = signbit(xv[i][j]) ? 8 : 0;
+                        sq[j] = xv[i][j] * xv[i][j];
+                    }
+                    r6[i] = r4[i] = or_tree(sq, 16);
+                } else {
+                    s6 = or_fwd46_candidate(xv[i], a, g, 6.0f, c6[i], &r6[i]);
+                    s4 = or_fwd46_candidate(xv[i], a, g, 4.0f, c4[i], &r4[i]);
+                }
+            }
+            float e6 = or_tree(r6, 16), e4 = or_tree(r4, 16);
+            int pick4 = !zero_tensor && (e4 < e6);
+            for (int i = 0; i < 16; i++) {
+                int64_t r = rb * 16 + i;
+                uint8_t *cc = pick4 ? c4[i] : c6[i];
+                for (int j = 0; j < 8; j++)
+                    codes[r * (C / 2) + q * 8 + j] = (uint8_t)(cc[2 * j] | (cc[2 * j + 1] << 4));
+                scales[r * G + q] = pick4 ? s4 : s6;
+            }
+            if (choice) choice[rb * G + q] = pick4 ? 4 : 6;
+            if (err6) err6[rb * G + q] = e6;
+            if (err4) err4[rb * G + q] = e4;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ backward: MS-EDEN */
 /* Stage 1 of MS-EDEN over rows [r0, r1) of a bf16 [R][C] matrix grouped along C (C a multiple
  * of 128).  Per 128-block ([QII-tg] "Method", item 1; [QII-ru] "Unbiased quantization with MS-EDEN"):
