@@ -44,6 +44,7 @@ BYTES_FWD46 = 2 + 2 + 0.5 + 1 / 16            # max pass read, quantize read, co
 BYTES_MSED_ONE = 2 + 0.5 + 0.25 + 0.25 + 1 / 16  # read, codes, pre-scale write + read, scales
 BYTES_MSED_BOTH = 2 + 2 * (0.5 + 0.25 + 0.25 + 1 / 16)
 BYTES_FUSED_X = 2 + 2 + (0.5 + 1 / 16) + (0.5 + 0.25 + 0.25 + 1 / 16)   # max read, read, both views
+BYTES_FWD46_SQ = 2 + 2 + 2 * (0.5 + 1 / 16)   # max read, read, row and column views
 
 
 def peaks():
@@ -332,6 +333,40 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return dict(M=M, K=K, N=N, max_ms=max_ms, per=per, status=status, clocks=clk.summary(), e2e=e2e)
 
 
+def run_op(args):
+    """--op fwd46_sq: the square-block weight quantizer on the config's W [N][K] (both views),
+    timed alone with CUDA events (two W inputs alternate; W is smaller than L2, so the second
+    pass of each call reads what the max pass left in L2)."""
+    import torch
+    from nvfp4_quantized_b200 import build as qbuild
+    from nvfp4_quantized_b200 import qt2 as Q, synth
+    qbuild.build()
+    dev = torch.device("cuda", 0)
+    M, K, N = synth.SHAPES[args.config]
+    ws_ = [synth.linear_inputs(args.config, seed=10 * i, device=dev)[1] for i in range(2)]
+    vr, vc = Q.alloc_view(N, K, dev), Q.alloc_view(K, N, dev)
+    ws = Q.alloc_workspace(Q.qt2_quant_fwd46_sq_workspace_size(N, K), dev)
+    st = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        Q.qt2_quant_fwd46_sq(ws_[i % 2], N, K, K, vr, vc, ws, ws.numel(), st)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for i in range(args.steps):
+        Q.qt2_quant_fwd46_sq(ws_[i % 2], N, K, K, vr, vc, ws, ws.numel(), st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    assert Q.qt2_device_status(st) == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    gbs = N * K * BYTES_FWD46_SQ / (ms * 1e-3) / 1e9
+    pk = peaks()
+    print(json.dumps({"op": "qt2_quant_fwd46_sq", "metric": "square-block quantizer GB/s (algorithmic bytes)",
+                      "value": gbs, "unit": "GB/s", "ms_per_call": ms, "hbm_frac": gbs / pk["hbm_gbs"],
+                      "steps": args.steps, "warmup": args.warmup,
+                      "config": {"tensor": f"W {N}x{K} bf16", "views": "row [N][K] and column [K][N]"}}),
+          flush=True)
+
+
 def cpu_baseline(config: str, tokens: int = 256):
     """The oracle, as it stands, on a bounded sample of the workload: the full step restricted
     to `tokens` rows of X and dY (W in full).  Returns (TFLOP/s, seconds, cores, sample)."""
@@ -367,9 +402,13 @@ def main():
                     help="fused: X's forward and column views from one read (qt2_quant_fwd46_msedEN_col) and "
                          "W's column view made once and reused by every step, as micro-batches of one "
                          "optimizer step")
+    ap.add_argument("--op", choices=["fwd46_sq"], default=None,
+                    help="time one library call alone instead of the layer step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.op:
+        return run_op(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

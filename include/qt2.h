@@ -103,6 +103,26 @@ QT2_API qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t col
                            size_t ws_bytes, qt2_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Square-block forward quantizer: one E4M3 scale per 16x16 block ([QII-tg] "Method": the pages
+ * compare 16x16 blocks with the 1x16 groups the method keeps for their lower error; with square
+ * blocks a weight and its transpose are the same quantization, so one pass serves both of its
+ * GEMM operand views).  x_bf16 [rows][cols] (ld):
+ *   row_out: view with R = rows, C = cols (groups along cols; the 16 rows of a block repeat its
+ *            scale), e.g. W [N][K] for the forward GEMM;
+ *   col_out: view of x^T with R = cols, C = rows: the same quantized values transposed, e.g.
+ *            W^T [K][N] for a dgrad GEMM with unrotated operands.
+ * Per block: a = max|x| over its 256 elements; for k = 6 and 4 the scale E4M3_RNE(a/(g*k)) and
+ * the RTN codes of every element; the block's squared error is the balanced tree over its 256
+ * elements in row-major order; keep 4 iff its error is smaller (a tie keeps 6); g = A/1792 as
+ * qt2_quant_fwd46.  Bit-identical to the reference algorithm.
+ * Workspace: at least qt2_quant_fwd46_sq_workspace_size() bytes, 16-byte aligned.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_fwd46_sq_workspace_size(int64_t rows, int64_t cols, size_t *bytes);
+QT2_API qt2_status qt2_quant_fwd46_sq(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                      const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                                      size_t ws_bytes, qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * Backward quantizer MS-EDEN (MicroScaling EDEN).  [QII-tg] "Method": a random Hadamard rotation
  * and a factor <x,x>/<Q(Rx),Rx> (EDEN), plus stochastic rounding of the FP8 scales;
  * [QII-th] "Question 1": fixed 128-element rotation groups, one shared rotation and seed, and

@@ -53,6 +53,15 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaGetLastError();
 }
 
+cudaError_t launch_fwd46_sq(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
+                            DevView row, DevView col, cudaStream_t s) {
+    const int64_t pairs = (R / 16) * (C / 16) / 2;   // two 16x16 blocks per warp
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((pairs + 7) / 8, (int64_t)sm_count() * 16));
+    fwd46_sq_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, R, C, ld, amax_word, row.codes, row.scales, row.tensor_scale,
+                                                     col.codes, col.scales, col.tensor_scale);
+    return cudaGetLastError();
+}
+
 template <int MODE, bool ROW, bool COL>
 static cudaError_t launch_rot_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed,
                                       const RotViews &out, cudaStream_t s) {
@@ -321,6 +330,15 @@ qt2_status fwd46_msed_col_enqueue(const void *x, int64_t rows, int64_t cols, int
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     return from_cuda(
         launch_msed_finalize(P_col, cols, rows, amax + 1, tid_col, col, nullptr, 0, 0, nullptr, 0, col, seed, s));
+}
+
+qt2_status fwd46_sq_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView row, DevView col,
+                            uint32_t *amax, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
+    if (e != cudaSuccess) return QT2_ERR_CUDA;
+    return from_cuda(launch_fwd46_sq(static_cast<const uint16_t *>(x), rows, cols, ld, amax, row, col, s));
 }
 
 qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *amax,
@@ -678,6 +696,27 @@ qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t 
     if ((st = gemm_enqueue(L.dy_row, L.w_col, M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK) return st;
     // wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
     return gemm_enqueue(L.dy_col, L.x_col, N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
+}
+
+qt2_status qt2_quant_fwd46_sq_workspace_size(int64_t rows, int64_t cols, size_t *bytes) {
+    if (!bytes) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(rows) || !dim_ok(cols)) return QT2_ERR_SHAPE;
+    *bytes = kWsAlign;
+    return QT2_OK;
+}
+
+qt2_status qt2_quant_fwd46_sq(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                              const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
+                              size_t ws_bytes, qt2_stream_t stream) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!view_ok(col_out)) return col_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < kWsAlign) return QT2_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QT2_ERR_ALIGN;
+    if ((st = check_device()) != QT2_OK) return st;
+    return fwd46_sq_enqueue(x_bf16, rows, cols, ld, dev_view(row_out), dev_view(col_out),
+                            static_cast<uint32_t *>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 
 qt2_status qt2_quant_fwd46_msedEN_col_workspace_size(int64_t rows, int64_t cols, size_t *bytes) {

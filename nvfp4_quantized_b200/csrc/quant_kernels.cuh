@@ -239,6 +239,96 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
 }
 
 // ---------------------------------------------------------------------------------------------
+// Square-block forward quantizer: one E4M3 scale per 16x16 block, so the quantized matrix and its
+// transpose are one quantization and a single pass writes both operand views of a weight
+// ([QII-tg] "Method": the pages weigh 16x16 blocks against the 1x16 groups they keep).  The
+// forward quantizer's steps with the block in place of the group: a = max|x| of the block, for
+// k = 6, 4 the scale E4M3_RNE(a/(g*k)) and RTN codes, block error = tree of the 16 rows' trees,
+// keep 4 iff its error is smaller.
+// Lane j of a half-warp holds row j of a block (16 elements, one 32-byte load); the half-warp's
+// xor-shuffles over lane bits 0..3 give the block max and the row-error tree in the reference
+// order (level 1 pairs rows 2i and 2i+1).  Two blocks per warp (adjacent along C).  The column
+// view ([C][R]) is the transpose: lane j gathers nibble j of every row of its half.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+    return __shfl_xor_sync(0xFFFFFFFFu, (unsigned long long)v, m);
+}
+
+__global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
+                                                       int64_t ld, const uint32_t *__restrict__ amax_word,
+                                                       uint8_t *__restrict__ row_codes, uint8_t *__restrict__ row_scales,
+                                                       float *__restrict__ row_g, uint8_t *__restrict__ col_codes,
+                                                       uint8_t *__restrict__ col_scales, float *__restrict__ col_g) {
+    const float g = fwd46_tensor_scale(amax_word);
+    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *row_g = g;
+        *col_g = g;
+    }
+    __shared__ float tab_d[128], tab_r[128];
+    fwd46_tables(g, tab_d, tab_r);
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, j = lane & 15;
+    const int64_t QB = C >> 4;                              // blocks along C (even)
+    const int64_t pairs = (R >> 4) * QB / 2;                // warp work items: two adjacent blocks
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < pairs; p += nwarps) {
+        const int64_t bi = 2 * p + (lane >> 4);
+        const int64_t rb = bi / QB, q = bi - rb * QB;
+        const int64_t r = rb * 16 + j;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + q * 16);
+        const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint64_t X[8];
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+            X[i] = f2(lo, hi);
+            a = fmaxf(a, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, m));   // block max (exact)
+        const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
+        uint32_t c6[2], c4[2];
+        float e6[8], e4[8];
+        fwd46_candidate(X, s6, c6, e6);
+        fwd46_candidate(X, s4, c4, e4);
+        uint64_t t[8];   // (candidate 6, candidate 4): the row's tree, then the rows' tree
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
+#pragma unroll
+        for (int sz = 8; sz > 1; sz >>= 1) {
+#pragma unroll
+            for (int i = 0; i < sz / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
+        }
+        uint64_t tb = t[0];
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1) tb = f2_add(tb, shfl_xor_u64(tb, m));   // addition commutes: same bits
+        float err6, err4;
+        f2_split(tb, err6, err4);
+        const bool pick4 = err4 < err6;                     // a tie keeps the full grid
+        const uint32_t code0 = pick4 ? c4[0] : c6[0], code1 = pick4 ? c4[1] : c6[1];
+        const uint32_t sc = pick4 ? s4.code : s6.code;
+        // row view: row r, group q
+        *reinterpret_cast<uint2 *>(row_codes + r * (C >> 1) + q * 8) = make_uint2(code0, code1);
+        row_scales[sf_offset(r, q, C)] = (uint8_t)sc;
+        // column view: row 16q + j of the transpose, group rb; nibble i = element (16rb + i, 16q + j)
+        const uint64_t mine = ((uint64_t)code1 << 32) | code0;
+        uint64_t tr = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint64_t other = __shfl_sync(0xFFFFFFFFu, (unsigned long long)mine, (lane & 16) | i);
+            tr |= ((other >> (4 * j)) & 0xFull) << (4 * i);
+        }
+        const int64_t cr = q * 16 + j;
+        *reinterpret_cast<uint2 *>(col_codes + cr * (R >> 1) + rb * 8) = make_uint2((uint32_t)tr, (uint32_t)(tr >> 32));
+        col_scales[sf_offset(cr, rb, R)] = (uint8_t)sc;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 // The 128 rotation signs of one backward call: bit i of Philox(seed, tensor id 0) word i/32 set
 // -> negate element i of every 128-block ([QII-th] "Question 1": one shared rotation and seed).
 // ---------------------------------------------------------------------------------------------

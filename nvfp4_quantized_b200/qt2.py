@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
                 "qt2_linear_fwd": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
                 "qt2_linear_bwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_bwd": (i32, [vp, vp, vp, i64, i64, i64, u64, vp, vp, i32, vp, sz, vp]),
+                "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
+                "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
                 "qt2_quant_fwd46_msedEN_col_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_msedEN_col": (i32, [vp, i64, i64, i64, u64, u32, pv, pv, vp, sz, vp]),
                 "qt2_linear_bwd_views_workspace_size": (i32, [i64, i64, i64, psz]),
@@ -284,3 +286,16 @@ def qt2_linear_bwd_views(dy: torch.Tensor, M: int, K: int, N: int, seed: int, x_
     _check("qt2_linear_bwd_views", lib().qt2_linear_bwd_views(
         _ptr(dy), M, K, N, seed, ctypes.byref(xc), ctypes.byref(wc), _ptr(dx), _ptr(dw), dw_dtype, _ptr(workspace),
         ws_bytes, _stream(stream)))
+
+
+def qt2_quant_fwd46_sq_workspace_size(rows: int, cols: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("qt2_quant_fwd46_sq_workspace_size", lib().qt2_quant_fwd46_sq_workspace_size(rows, cols, ctypes.byref(n)))
+    return n.value
+
+
+def qt2_quant_fwd46_sq(x: torch.Tensor, rows: int, cols: int, ld: int, row_out: View, col_out: View,
+                       workspace: torch.Tensor, ws_bytes: int, stream=None) -> None:
+    r, c = row_out.c(), col_out.c()
+    _check("qt2_quant_fwd46_sq", lib().qt2_quant_fwd46_sq(_ptr(x), rows, cols, ld, ctypes.byref(r), ctypes.byref(c),
+                                                          _ptr(workspace), ws_bytes, _stream(stream)))

@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 19
+    assert len(names) == 21
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -94,6 +94,11 @@ def test_host_validation_codes(L):
     assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(v), 0x40000, 16, None) == qt2.QT2_ERR_WORKSPACE
     assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(_view(scales=0x20004)), 0x40000, 1 << 20,
               None) == qt2.QT2_ERR_ALIGN
+    sq = L.qt2_quant_fwd46_sq
+    assert sq(0x1000, 128, 128, 128, None, R(v), 0x40000, 256, None) == qt2.QT2_ERR_INVALID_ARG
+    assert sq(0x1000, 128, 200, 200, R(v), R(v), 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
+    assert sq(0x1000, 128, 128, 128, R(v), R(v), 0x40000, 8, None) == qt2.QT2_ERR_WORKSPACE
+    assert sq(0x1002, 128, 128, 128, R(v), R(v), 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
     bv = L.qt2_linear_bwd_views
     assert bv(0x1000, 128, 128, 128, 0, None, R(v), 0x4000, 0x5000, 1, 0x6000, 1 << 30, None) == \
         qt2.QT2_ERR_INVALID_ARG
