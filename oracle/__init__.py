@@ -192,21 +192,35 @@ class View:
     def shape(self):
         return self.codes.shape[0], self.codes.shape[1] * 2
 
+    def row_g(self) -> np.ndarray:
+        """The tensor scale of every row: g itself, or for a view with one scale per block of
+        `row_block` rows (the CTA-local variant) that block's entry of the array g."""
+        R = self.shape[0]
+        if np.ndim(self.g) == 0:
+            return np.full(R, self.g, np.float32)
+        return np.repeat(np.asarray(self.g, np.float32), self.row_block)
+
     def dequant(self) -> np.ndarray:
-        """xhat = val(code) * E4M3(scale) * g, fp64."""
+        """xhat = val(code) * E4M3(scale) * g (g of the row's block for a CTA-local view), fp64
+        (the products of a 2-bit, a 4-bit and a 24-bit significand are exact in any order)."""
         R, C = self.shape
         out = np.empty((R, C), dtype=np.float64)
-        _rows(lambda r0, r1: lib().or_dequant(_p(self.codes), _p(self.scales), R, C, float(self.g), r0, r1, _p(out)), R)
-        return out
+        if np.ndim(self.g) == 0:
+            _rows(lambda r0, r1: lib().or_dequant(_p(self.codes), _p(self.scales), R, C, float(self.g), r0, r1,
+                                                  _p(out)), R)
+            return out
+        _rows(lambda r0, r1: lib().or_dequant(_p(self.codes), _p(self.scales), R, C, 1.0, r0, r1, _p(out)), R)
+        return out * self.row_g().astype(np.float64)[:, None]
 
     def dequant_rows(self, rows) -> np.ndarray:
         """Dequantized rows (fp64) of the given row indices only."""
         R, C = self.shape
+        rg = self.row_g()
         out = np.empty((len(rows), C), dtype=np.float64)
         for i, r in enumerate(rows):
             row = np.empty(C, dtype=np.float64)
-            lib().or_dequant_row(_p(self.codes), _p(self.scales), R, C, float(self.g), int(r), _p(row))
-            out[i] = row
+            lib().or_dequant_row(_p(self.codes), _p(self.scales), R, C, 1.0, int(r), _p(row))
+            out[i] = row * float(rg[r])
         return out
 
 
@@ -226,6 +240,28 @@ def fwd46(x, A: float | None = None) -> View:
                                              _p(e6), _p(e4)), R)
     return View(codes, scales, lib().or_fwd46_tensor_scale(A), amax=np.float32(A), choice=choice,
                 err6=e6, err4=e4)
+
+
+def fwd46_local(x, row_block: int = 128) -> View:
+    """CTA-local forward quantizer ([FAF] "the speed-up is lost between the matmuls": the
+    CTA-local NVFP4 variant keeps the scale dependency inside a thread block -- rows and columns
+    get their own corrections, constant during the summation and applied after it -- so no
+    block waits for the tensor-wide maximum, at the price of a different numeric contract).
+    Per block of `row_block` rows: A_b = max|x| over the block (all columns), then the forward
+    quantizer of those rows with g_b = A_b/1792.  The view's g is the array of the g_b."""
+    b = _bf16_bits(x)
+    R, C = b.shape
+    assert R % row_block == 0
+    codes = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    choice = np.zeros((R, C // 16), np.uint8)
+    gs = np.empty(R // row_block, np.float32)
+    for blk in range(R // row_block):
+        r0, r1 = blk * row_block, (blk + 1) * row_block
+        A_b = amax_bf16(b[r0:r1])
+        lib().or_fwd46_rows(_p(b), R, C, A_b, r0, r1, _p(codes), _p(scales), _p(choice), None, None)
+        gs[blk] = lib().or_fwd46_tensor_scale(A_b)
+    return View(codes, scales, gs, row_block=row_block, choice=choice)
 
 
 def transpose_codes(codes: np.ndarray) -> np.ndarray:
