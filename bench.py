@@ -38,6 +38,8 @@ KERNELS_PER_STEP = 13   # per step: 2 max + 2 fwd46 + 3 GEMM + 3 MS-EDEN produce
 # --schedule fused: X max + X's two views in one pass + its finalize, W max + fwd46, dY MS-EDEN +
 # finalize, 3 GEMMs (W's column view is made once, before the timed steps)
 KERNELS_PER_STEP_FUSED = 10
+# --schedule local: one CTA-local quantizer launch each for X and W, then as the default schedule
+KERNELS_PER_STEP_LOCAL = 11
 
 # Algorithmic bytes per input element of each quantizer call (reads + writes the method needs).
 BYTES_FWD46 = 2 + 2 + 0.5 + 1 / 16            # max pass read, quantize read, codes, scales
@@ -191,9 +193,41 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         Q.qt2_gemm_nvfp4(v_dy_col, v_x_col, N, K, M, 2.0 ** -7, dw, Q.QT2_DTYPE_F32, K, stream)
         mark(6)
 
+    local = args.schedule == "local"
+    if local:
+        vxl, vwl = Q.alloc_view_local(M, K, dev), Q.alloc_view_local(N, K, dev)
+
+    def step_local(i, ev=None):
+        x, w, dy = sets[i % 2]
+        seed = 0x5EED0000 + i
+
+        def mark(j):
+            if ev is not None:
+                ev[j].record(stream)
+        mark(0)
+        Q.qt2_quant_fwd46_local(x, M, K, K, vxl, stream)
+        mark(1)
+        Q.qt2_quant_fwd46_local(w, N, K, K, vwl, stream)
+        mark(2)
+        Q.qt2_gemm_nvfp4_local(vxl, vwl, M, N, K, 1.0, y, Q.QT2_DTYPE_BF16, N, stream)
+        mark(3)
+        Q.qt2_quant_msedEN(dy, M, N, N, BOTH, seed, Q.QT2_TID_DY_ROW, Q.QT2_TID_DY_COL, v_dy_row, v_dy_col, ws_dy,
+                           ws_dy.numel(), stream)
+        mark(4)
+        Q.qt2_quant_msedEN(w, N, K, K, COL, seed, 0, Q.QT2_TID_W_COL, None, v_w_col, ws_w, ws_w.numel(), stream)
+        mark(5)
+        Q.qt2_quant_msedEN(x, M, K, K, COL, seed, 0, Q.QT2_TID_X_COL, None, v_x_col, ws_x, ws_x.numel(), stream)
+        mark(6)
+        Q.qt2_gemm_nvfp4(v_dy_row, v_w_col, M, K, N, 2.0 ** -7, dx, Q.QT2_DTYPE_BF16, K, stream)
+        mark(7)
+        Q.qt2_gemm_nvfp4(v_dy_col, v_x_col, N, K, M, 2.0 ** -7, dw, Q.QT2_DTYPE_F32, K, stream)
+        mark(8)
+
     def step(i, ev=None):
         if fused:
             return step_fused(i, ev)
+        if local:
+            return step_local(i, ev)
         x, w, dy = sets[i % 2]
         seed = 0x5EED0000 + i
 
@@ -398,10 +432,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--cpu-tokens", type=int, default=2048)
-    ap.add_argument("--schedule", choices=["separate", "fused"], default="separate",
+    ap.add_argument("--schedule", choices=["separate", "fused", "local"], default="separate",
                     help="fused: X's forward and column views from one read (qt2_quant_fwd46_msedEN_col) and "
                          "W's column view made once and reused by every step, as micro-batches of one "
-                         "optimizer step")
+                         "optimizer step; local: the forward with CTA-local scales (qt2_quant_fwd46_local, "
+                         "qt2_gemm_nvfp4_local), a different numeric contract")
     ap.add_argument("--op", choices=["fwd46_sq"], default=None,
                     help="time one library call alone instead of the layer step")
     args = ap.parse_args()
@@ -504,7 +539,8 @@ def main():
                        "hbm_frac": quant_bytes / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                        "peak_gbs": pk["hbm_gbs"], "ms_per_step": quant_ms},
         "kernels": kernels,
-        "gpu_launches": (KERNELS_PER_STEP_FUSED if args.schedule == "fused" else KERNELS_PER_STEP) * args.steps,
+        "gpu_launches": {"fused": KERNELS_PER_STEP_FUSED, "local": KERNELS_PER_STEP_LOCAL}.get(
+            args.schedule, KERNELS_PER_STEP) * args.steps,
         "clocks": r["clocks"],
         "device_status": r["status"],
     }
@@ -525,6 +561,9 @@ def run_names(schedule: str):
     """The calls of one step, in order (each is timed with CUDA events)."""
     if schedule == "fused":
         return ["fused_x_views", "fwd46_w", "gemm_fwd", "msed_dy_both", "gemm_dgrad", "gemm_wgrad"]
+    if schedule == "local":
+        return ["fwd46_local_x", "fwd46_local_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col",
+                "gemm_dgrad", "gemm_wgrad"]
     return ["fwd46_x", "fwd46_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col", "gemm_dgrad", "gemm_wgrad"]
 
 
@@ -532,7 +571,8 @@ def quant_bytes_per_call(M: int, K: int, N: int):
     """Algorithmic bytes of each quantizer call of a step."""
     return {"fwd46_x": M * K * BYTES_FWD46, "fwd46_w": N * K * BYTES_FWD46, "msed_dy_both": M * N * BYTES_MSED_BOTH,
             "msed_w_col": N * K * BYTES_MSED_ONE, "msed_x_col": M * K * BYTES_MSED_ONE,
-            "fused_x_views": M * K * BYTES_FUSED_X}
+            "fused_x_views": M * K * BYTES_FUSED_X, "fwd46_local_x": M * K * BYTES_FWD46,
+            "fwd46_local_w": N * K * BYTES_FWD46}
 
 
 if __name__ == "__main__":

@@ -103,6 +103,24 @@ QT2_API qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t col
                            size_t ws_bytes, qt2_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * CTA-local forward quantizer and GEMM ([FAF] "the speed-up is lost between the matmuls": in
+ * the CTA-local NVFP4 variant the scale dependency stays inside one thread block; rows and
+ * columns get their own corrections, constant over the summation and applied after it, so no
+ * block waits for the tensor-wide maximum; the numeric contract differs from global NVFP4).
+ * qt2_quant_fwd46_local: x_bf16 [rows][cols] (ld) -> a view like qt2_quant_fwd46's except
+ *   that row_out->tensor_scale points to rows/128 floats: block b of 128 rows is quantized with
+ *   g_b = A_b/1792, A_b = max|x| over its rows (g_b = 1 below 2^-100).  One launch, no
+ *   workspace, no tensor-wide reduction.
+ * qt2_gemm_nvfp4_local: as qt2_gemm_nvfp4 for two such views (a: M/128 scales, b: N/128):
+ *   c[m][n] = alpha * ga[m/128] * gb[n/128] * sum_k val(a)*sa * val(b)*sb.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_quant_fwd46_local(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                         const qt2_nvfp4_view *row_out, qt2_stream_t stream);
+QT2_API qt2_status qt2_gemm_nvfp4_local(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N,
+                                        int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
+                                        qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * Square-block forward quantizer: one E4M3 scale per 16x16 block ([QII-tg] "Method": the pages
  * compare 16x16 blocks with the 1x16 groups the method keeps for their lower error; with square
  * blocks a weight and its transpose are the same quantization, so one pass serves both of its

@@ -2,7 +2,8 @@
 //
 // "Quartet II ... MS-EDEN" Thai translation (itsolotime.com archives 22992), abstract and §1:
 // NVFP4 is multiplied natively by Blackwell tensor cores.  Same contract as gemm_kernel.cuh:
-// C = alpha * gA * gB * sum_k val(A) sA * val(B) sB, both operands K-major, fp32 accumulation.
+// C = alpha * gA * gB * sum_k val(A) sA * val(B) sB, both operands K-major, fp32 accumulation
+// (with `local`, gA and gB are per-128-row arrays: the row's and the column's block scale).
 //
 // Why a pair: with one SM per 128x256 tile, every SM streams 216 KB of operands per K = 256
 // step from L2.  A CTA pair computes a 256x256 tile with one tcgen05.mma.cta_group::2: each SM
@@ -49,20 +50,6 @@
 namespace qt2 {
 
 // ------------------------------------------------------------------ cluster / pair wrappers
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Shared-memory address of the same variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -93,11 +80,6 @@ __device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
                      bar),
                  "h"(both)
                  : "memory");
-}
-__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-    return v;
 }
 // 32 lanes x 32 bits x 16 columns: thread t writes lane (quadrant*32 + t), columns [col, col+16).
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -182,7 +164,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const float *__restrict__ gA, const float *__restrict__ gB, float alpha,
-                           void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype) {
+                           void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype, int local) {
     using Cfg = Gemm2Cfg;
     constexpr int S = Cfg::kStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -323,7 +305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         const int quad = warp & 3, ew = warp - Cfg::kEpiWarp0;
         const int cb = (ew >> 2) * 128;   // this warp's 128 of the tile's 256 columns
         const uint32_t acc_empty_leader = mapa_shared(acc_empty, 0);
-        const float sc = alpha * (*gA) * (*gB);
         const int64_t row_bytes = ldc * (c_dtype == QT2_DTYPE_F32 ? 4 : 2);
         const bool wide = (reinterpret_cast<uintptr_t>(Cout) & 31) == 0 && (row_bytes & 31) == 0;
         for (int t_iter = 0; t_iter < my_tiles; ++t_iter) {
@@ -333,6 +314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             const int pm = tile / num_pn, pn = tile - pm * num_pn;
             const int64_t row = (int64_t)pm * 256 + rank * 128 + quad * 32 + lane;
             const int64_t col = (int64_t)pn * 256 + cb;
+            // tensor scales: one each, or (CTA-local views) one per 128 rows of A and of B
+            const float sc = local ? alpha * gA[pm * 2 + (int)rank] * gB[pn * 2 + (cb >> 7)] : alpha * (*gA) * (*gB);
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + cb;
             // All 128 columns into registers first, then release the accumulator, so the next
             // tile's MMAs overlap the scaling and the stores.

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb, const float *__restrict__ gA,
                       const float *__restrict__ gB, float alpha, void *__restrict__ Cout, int64_t ldc, int K,
-                      int c_dtype) {
+                      int c_dtype, int local) {
     using Cfg = GemmCfg<BN>;
     constexpr int S = Cfg::kStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -142,11 +142,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool acc_ok = mbar_wait_warp(accum_bar, 0);
     tc_fence_after();
     if (acc_ok) {
-        const float sc = alpha * (*gA) * (*gB);
         const int64_t row = m0 + warp * 32 + lane;
         const uint32_t t_row = t_acc + ((uint32_t)(warp * 32) << 16);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
+            // tensor scales: one each, or (CTA-local views) one per 128 rows of A and of B
+            const float sc = local ? alpha * gA[m0 >> 7] * gB[(n0 + c) >> 7] : alpha * (*gA) * (*gB);
             uint32_t v[16];
             tmem_ld_32x32b_x16(t_row + c, v);
             tmem_ld_wait();

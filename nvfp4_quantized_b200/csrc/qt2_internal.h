@@ -35,13 +35,15 @@ cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, boo
 cudaError_t launch_msed_finalize(const float *P_a, int64_t R_a, int64_t C_a, const uint32_t *amax_a, uint32_t tid_a,
                                  DevView out_a, const float *P_b, int64_t R_b, int64_t C_b, const uint32_t *amax_b,
                                  uint32_t tid_b, DevView out_b, uint64_t seed, cudaStream_t s);
+// local = 1: a.tensor_scale / b.tensor_scale are per-128-row arrays (CTA-local views)
 cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
-                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s);
+                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s,
+                              int local = 0);
 
 cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
                                    const CUtensorMap &tmSFB, DevView a, DevView b, int64_t M,
                                    int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
-                                   cudaStream_t s);
+                                   cudaStream_t s, int local = 0);
 
 // 2D tensor map for TMA (no multicast anywhere in this library).
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,

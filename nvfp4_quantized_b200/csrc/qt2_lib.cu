@@ -53,6 +53,12 @@ cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaGetLastError();
 }
 
+cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t ld, DevView out, cudaStream_t s) {
+    fwd46_local_kernel<<<(unsigned)(R / 128 * kLocalCluster), kLocalThreads, 0, s>>>(x, R, C, ld, out.codes,
+                                                                                     out.scales, out.tensor_scale);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_fwd46_sq(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
                             DevView row, DevView col, cudaStream_t s) {
     const int64_t pairs = (R / 16) * (C / 16) / 2;   // two 16x16 blocks per warp
@@ -140,7 +146,7 @@ cudaError_t launch_msed_finalize(const float *P_a, int64_t R_a, int64_t C_a, con
 template <int BN>
 static cudaError_t launch_gemm_bn(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
                                   int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, int local) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -150,20 +156,21 @@ static cudaError_t launch_gemm_bn(const CUtensorMap &tmA, const CUtensorMap &tmB
     if (attr_err != cudaSuccess) return attr_err;
     dim3 grid((unsigned)(N / BN), (unsigned)(M / kGemmBM));
     gemm_nvfp4_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, s>>>(
-        tmA, tmB, a.scales, b.scales, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)K, c_dtype);
+        tmA, tmB, a.scales, b.scales, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)K, c_dtype, local);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_nvfp4(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
-                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s) {
-    if (N % 256 == 0) return launch_gemm_bn<256>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
-    return launch_gemm_bn<128>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s);
+                              int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc, cudaStream_t s,
+                              int local) {
+    if (N % 256 == 0) return launch_gemm_bn<256>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s, local);
+    return launch_gemm_bn<128>(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s, local);
 }
 
 cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmSFA,
                                    const CUtensorMap &tmSFB, DevView a, DevView b, int64_t M,
                                    int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, int local) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -174,7 +181,8 @@ cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tm
     const int64_t tiles = (M / 256) * (N / 256);
     const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count() / 2));
     gemm_nvfp4_pair_kernel<<<(unsigned)(2 * clusters), Gemm2Cfg::kThreads, Gemm2Cfg::kSmemBytes, s>>>(
-        tmA, tmB, tmSFA, tmSFB, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype);
+        tmA, tmB, tmSFA, tmSFB, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype,
+        local);
     return cudaGetLastError();
 }
 
@@ -352,7 +360,7 @@ qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, 
 }
 
 qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, float alpha, void *c, int c_dtype,
-                        int64_t ldc, cudaStream_t s) {
+                        int64_t ldc, cudaStream_t s, int local = 0) {
     CUtensorMap tmA, tmB;
     if (M % 256 == 0 && N % 256 == 0) {
         // pair kernel: 128-row code boxes per SM, scale atoms as rows of K/64 512-byte atoms
@@ -366,7 +374,8 @@ qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, f
             !encode_tmap_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT64, b.scales, (uint64_t)K, (uint64_t)N / 128,
                             (uint64_t)K * 8, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
             return QT2_ERR_CUDA;
-        return from_cuda(launch_gemm_nvfp4_pair(tmA, tmB, tmSFA, tmSFB, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
+        return from_cuda(
+            launch_gemm_nvfp4_pair(tmA, tmB, tmSFA, tmSFB, a, b, M, N, K, alpha, c, c_dtype, ldc, s, local));
     }
     const int bn = (N % 256 == 0) ? 256 : 128;
     if (!encode_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
@@ -374,7 +383,7 @@ qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, f
         !encode_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b.codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
                         (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B))
         return QT2_ERR_CUDA;
-    return from_cuda(launch_gemm_nvfp4(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s));
+    return from_cuda(launch_gemm_nvfp4(tmA, tmB, a, b, M, N, K, alpha, c, c_dtype, ldc, s, local));
 }
 
 // Views carved from a workspace: codes, scales, tensor scale.
@@ -696,6 +705,32 @@ qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t 
     if ((st = gemm_enqueue(L.dy_row, L.w_col, M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK) return st;
     // wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
     return gemm_enqueue(L.dy_col, L.x_col, N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
+}
+
+qt2_status qt2_quant_fwd46_local(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                 const qt2_nvfp4_view *row_out, qt2_stream_t stream) {
+    qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
+    if (st != QT2_OK) return st;
+    if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
+    if ((st = check_device()) != QT2_OK) return st;
+    return from_cuda(launch_fwd46_local(static_cast<const uint16_t *>(x_bf16), rows, cols, ld, dev_view(row_out),
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qt2_status qt2_gemm_nvfp4_local(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,
+                                float alpha, void *c, int c_dtype, int64_t ldc, qt2_stream_t stream) {
+    if (!a || !b || !c) return QT2_ERR_INVALID_ARG;
+    if (c_dtype != QT2_DTYPE_BF16 && c_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
+    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K) || ldc < N) return QT2_ERR_SHAPE;
+    if (!view_ok(a) || !view_ok(b)) return (a->codes && a->scales && a->tensor_scale && b->codes && b->scales &&
+                                            b->tensor_scale)
+                                               ? QT2_ERR_ALIGN
+                                               : QT2_ERR_INVALID_ARG;
+    if (!aligned16(c) || ldc % 8 != 0) return QT2_ERR_ALIGN;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    return gemm_enqueue(dev_view(a), dev_view(b), M, N, K, alpha, c, c_dtype, ldc,
+                        reinterpret_cast<cudaStream_t>(stream), 1);
 }
 
 qt2_status qt2_quant_fwd46_sq_workspace_size(int64_t rows, int64_t cols, size_t *bytes) {

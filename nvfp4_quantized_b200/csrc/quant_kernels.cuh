@@ -239,6 +239,84 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
 }
 
 // ---------------------------------------------------------------------------------------------
+// CTA-local forward quantizer ([FAF] "the speed-up is lost between the matmuls": the CTA-local
+// NVFP4 variant keeps the scale dependency inside a thread block; rows and columns get their own
+// corrections, constant over the summation and applied after it).  Block b of 128 rows is
+// quantized exactly as fwd46_rows_kernel does with the tensor scale g_b = A_b/1792 of its own
+// max (1 below 2^-100) -- no grid-wide dependency, one launch.  A cluster of 4 CTAs owns a
+// block (32 rows each, so that 64-row weights still fill the GPU): each takes the max of its
+// rows, the four partial maxima meet through distributed shared memory, and each CTA then
+// quantizes its rows (their second read mostly hits L2).
+// ---------------------------------------------------------------------------------------------
+constexpr int kLocalCluster = 4;
+constexpr int kLocalThreads = 256;
+
+__global__ void __cluster_dims__(kLocalCluster, 1, 1) __launch_bounds__(kLocalThreads)
+    fwd46_local_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C, int64_t ld, uint8_t *__restrict__ codes,
+                       uint8_t *__restrict__ scales, float *__restrict__ g_blocks) {
+    (void)R;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t blk = (int64_t)blockIdx.x / kLocalCluster;
+    const int64_t r0 = blk * 128 + (int64_t)rank * 32;    // this CTA's 32 rows
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kWarps = kLocalThreads / 32;
+    // max |x| of the CTA's rows: bf16 magnitudes order like their bit patterns with the sign cleared
+    uint32_t m = 0;
+    const int64_t vec_per_row = C >> 3;
+    for (int rr = warp; rr < 32; rr += kWarps) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(x + (r0 + rr) * ld);
+#pragma unroll 4
+        for (int64_t v = lane; v < vec_per_row; v += 32) {
+            const uint4 w = row[v];
+            m = __vmaxu2(m, w.x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, w.w & 0x7FFF7FFFu);
+        }
+    }
+    __shared__ uint32_t wmax[kWarps];
+    __shared__ uint32_t cta_max;
+    const uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16) << 16);
+    if (lane == 0) wmax[warp] = bits;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int i = 0; i < kWarps; ++i) b = max(b, wmax[i]);
+        cta_max = b;
+    }
+    cluster_sync_all();   // every CTA's partial max is visible to its cluster
+    uint32_t bmax = 0;
+#pragma unroll
+    for (int c = 0; c < kLocalCluster; ++c) bmax = max(bmax, ld_shared_cluster_u32(mapa_shared(smem_u32(&cta_max), c)));
+    cluster_sync_all();   // no CTA leaves while a peer may still read its partial max
+    const float A = __uint_as_float(bmax);
+    const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
+    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    if (rank == 0 && threadIdx.x == 0) g_blocks[blk] = g;
+    __shared__ float tab_d[128], tab_r[128];
+    fwd46_tables(g, tab_d, tab_r);
+    __syncthreads();
+    // the CTA's groups, one per thread and round (4 consecutive lanes: one scale word)
+    const uint32_t G = (uint32_t)(C >> 4);
+    const uint32_t total = 32u * G;                    // a multiple of 256
+    for (uint32_t gi = threadIdx.x; gi < total; gi += kLocalThreads) {
+        const int64_t r = r0 + gi / G;
+        const uint32_t q = gi % G;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (int64_t)q * 16);
+        const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+        const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t code0, code1;
+        const uint32_t sc = fwd46_group(w, g6, g4, tab_d, tab_r, code0, code1);
+        *reinterpret_cast<uint2 *>(codes + r * (C >> 1) + (int64_t)q * 8) = make_uint2(code0, code1);
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
+        if ((lane & 3) == 0)
+            *reinterpret_cast<uint32_t *>(scales + sf_offset(r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Square-block forward quantizer: one E4M3 scale per 16x16 block, so the quantized matrix and its
 // transpose are one quantization and a single pass writes both operand views of a weight
 // ([QII-tg] "Method": the pages weigh 16x16 blocks against the 1x16 groups they keep).  The

@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
                 "qt2_linear_fwd": (i32, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
                 "qt2_linear_bwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_bwd": (i32, [vp, vp, vp, i64, i64, i64, u64, vp, vp, i32, vp, sz, vp]),
+                "qt2_quant_fwd46_local": (i32, [vp, i64, i64, i64, pv, vp]),
+                "qt2_gemm_nvfp4_local": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
                 "qt2_quant_fwd46_msedEN_col_workspace_size": (i32, [i64, i64, psz]),
@@ -299,3 +301,22 @@ def qt2_quant_fwd46_sq(x: torch.Tensor, rows: int, cols: int, ld: int, row_out: 
     r, c = row_out.c(), col_out.c()
     _check("qt2_quant_fwd46_sq", lib().qt2_quant_fwd46_sq(_ptr(x), rows, cols, ld, ctypes.byref(r), ctypes.byref(c),
                                                           _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def alloc_view_local(R: int, C: int, device="cuda") -> View:
+    """A view whose tensor scale is one float per 128 rows (CTA-local quantizer output)."""
+    v = alloc_view(R, C, device)
+    return View(v.codes, v.scales, torch.empty(R // 128, dtype=torch.float32, device=v.codes.device))
+
+
+def qt2_quant_fwd46_local(x: torch.Tensor, rows: int, cols: int, ld: int, row_out: View, stream=None) -> None:
+    r = row_out.c()
+    _check("qt2_quant_fwd46_local", lib().qt2_quant_fwd46_local(_ptr(x), rows, cols, ld, ctypes.byref(r),
+                                                                _stream(stream)))
+
+
+def qt2_gemm_nvfp4_local(a: View, b: View, M: int, N: int, K: int, alpha: float, c: torch.Tensor, c_dtype: int,
+                         ldc: int, stream=None) -> None:
+    ac, bc = a.c(), b.c()
+    _check("qt2_gemm_nvfp4_local", lib().qt2_gemm_nvfp4_local(ctypes.byref(ac), ctypes.byref(bc), M, N, K, alpha,
+                                                              _ptr(c), c_dtype, ldc, _stream(stream)))

@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 21
+    assert len(names) == 23
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -94,6 +94,14 @@ def test_host_validation_codes(L):
     assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(v), 0x40000, 16, None) == qt2.QT2_ERR_WORKSPACE
     assert fx(0x1000, 128, 128, 128, 1, 4, R(v), R(_view(scales=0x20004)), 0x40000, 1 << 20,
               None) == qt2.QT2_ERR_ALIGN
+    lq = L.qt2_quant_fwd46_local
+    assert lq(None, 128, 128, 128, R(v), None) == qt2.QT2_ERR_INVALID_ARG
+    assert lq(0x1000, 192, 128, 128, R(v), None) == qt2.QT2_ERR_SHAPE
+    assert lq(0x1000, 128, 128, 128, None, None) == qt2.QT2_ERR_INVALID_ARG
+    lg = L.qt2_gemm_nvfp4_local
+    assert lg(R(v), R(v), 128, 128, 128, 1.0, None, 0, 128, None) == qt2.QT2_ERR_INVALID_ARG
+    assert lg(R(v), R(v), 128, 128, 128, 1.0, 0x50000, 0, 64, None) == qt2.QT2_ERR_SHAPE
+    assert lg(R(v), R(v), 128, 128, 128, 1.0, 0x50008, 0, 128, None) == qt2.QT2_ERR_ALIGN
     sq = L.qt2_quant_fwd46_sq
     assert sq(0x1000, 128, 128, 128, None, R(v), 0x40000, 256, None) == qt2.QT2_ERR_INVALID_ARG
     assert sq(0x1000, 128, 200, 200, R(v), R(v), 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
