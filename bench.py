@@ -34,10 +34,12 @@ if ROOT not in sys.path:
 
 METRIC = "Quartet II linear fwd+bwd TFLOPS; quantizer GB/s; % of FP4/HBM roofline"
 UNIT = "TFLOP/s"
-KERNELS_PER_STEP = 13   # per step: 2 max + 2 fwd46 + 3 GEMM + 3 MS-EDEN producers + 3 finalize (dY views share one)
-# --schedule fused: X max + X's two views in one pass + its finalize, W max + fwd46, dY MS-EDEN +
+# per step: 2 fwd46 (max, grid barrier and quantization in one cooperative launch) + 3 GEMM + 3 MS-EDEN
+# producers + 3 finalize (dY's two views share one)
+KERNELS_PER_STEP = 11
+# --schedule fused: X max + X's two views in one pass + its finalize, W fwd46, dY MS-EDEN +
 # finalize, 3 GEMMs (W's column view is made once, before the timed steps)
-KERNELS_PER_STEP_FUSED = 10
+KERNELS_PER_STEP_FUSED = 9
 # --schedule local: one CTA-local quantizer launch each for X and W, then as the default schedule
 KERNELS_PER_STEP_LOCAL = 11
 

@@ -94,8 +94,10 @@ QT2_API qt2_status qt2_device_status(qt2_stream_t stream, int *code);
  * keeps k = 4 iff err_4 < err_6.  Results are bit-identical to the reference algorithm.
  * layout_mask must be QT2_LAYOUT_ROW (the forward GEMM consumes row views only); row_out
  * receives the view (R = rows, C = cols); col_out is ignored and may be NULL.
+ * One cooperative launch: its thread blocks merge the tensor max, meet at a grid barrier and
+ * then quantize (a tensor that fits in L2 is read from HBM once).
  * Workspace: at least qt2_quant_fwd46_workspace_size() bytes, 16-byte aligned; it holds the
- * tensor max and is overwritten.
+ * tensor max and the barrier's counter and is overwritten.
  * --------------------------------------------------------------------------------------- */
 QT2_API qt2_status qt2_quant_fwd46_workspace_size(int64_t rows, int64_t cols, size_t *bytes);
 QT2_API qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,

@@ -35,7 +35,7 @@
 // of the rotated view(s) and writes nothing else; kModeSr then quantizes with that tensor scale
 // (sr_vector).  kModeEden is MS-EDEN.  kModeFwdRowEdenCol gives both of X's views from one read
 // ([FAF]): the row warps quantize the tile's rows for the forward GEMM (RTN with the 4/6 choice,
-// as fwd46_rows_kernel, with the tensor max of X taken beforehand), the column warps produce the
+// as fwd46_coop_kernel, with the tensor max of X taken beforehand), the column warps produce the
 // MS-EDEN column view.
 #pragma once
 

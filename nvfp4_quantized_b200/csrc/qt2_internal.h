@@ -27,8 +27,6 @@ constexpr float kSrCutoff = 0x1p-6f;           // E4M3 scales below 2^-6 are rou
 // Kernel launchers (one translation unit: qt2_lib.cu).  Each returns the launch status.
 cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *amax_word,
                              cudaStream_t s);
-cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
-                              DevView out, cudaStream_t s);
 cudaError_t launch_msed_tiles(const CUtensorMap &tmap, int64_t R, int64_t C, bool do_row, bool do_col,
                               uint64_t seed, DevView row, DevView col, float *P_row, float *P_col,
                               uint32_t *amax_row, uint32_t *amax_col, cudaStream_t s);

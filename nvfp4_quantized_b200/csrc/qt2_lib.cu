@@ -44,13 +44,24 @@ cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld
     return cudaGetLastError();
 }
 
-cudaError_t launch_fwd46_rows(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
-                              DevView out, cudaStream_t s) {
+
+// The forward quantizer as one cooperative launch (words: 2 zeroed words, the max and the
+// barrier's arrivals).  The grid is every CTA that fits on the device at once.
+cudaError_t launch_fwd46_coop(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *words, DevView out,
+                              cudaStream_t s) {
+    static std::once_flag once;
+    static int per_sm = 0;
+    static cudaError_t occ_err = cudaSuccess;
+    std::call_once(once, [] { occ_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd46_coop_kernel, 256, 0); });
+    if (occ_err != cudaSuccess) return occ_err;
+    if (per_sm < 1) return cudaErrorLaunchOutOfResources;
     const int64_t groups = R * (C >> 4);
-    const int64_t blocks = std::min<int64_t>((groups + 255) / 256, (int64_t)sm_count() * 64);
-    fwd46_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, R, C, ld, amax_word, out.codes, out.scales,
-                                                       out.tensor_scale);
-    return cudaGetLastError();
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((groups + 255) / 256, (int64_t)per_sm * sm_count()));
+    uint8_t *codes = out.codes, *scales = out.scales;
+    float *ts = out.tensor_scale;
+    void *args[] = {(void *)&x, (void *)&R, (void *)&C, (void *)&ld, (void *)&words, (void *)&codes, (void *)&scales,
+                    (void *)&ts};
+    return cudaLaunchCooperativeKernel((const void *)fwd46_coop_kernel, dim3((unsigned)blocks), dim3(256), args, 0, s);
 }
 
 cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t ld, DevView out, cudaStream_t s) {
@@ -349,14 +360,13 @@ qt2_status fwd46_sq_enqueue(const void *x, int64_t rows, int64_t cols, int64_t l
     return from_cuda(launch_fwd46_sq(static_cast<const uint16_t *>(x), rows, cols, ld, amax, row, col, s));
 }
 
-qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *amax,
+// The forward quantizer: one cooperative launch (max, grid barrier, quantization).
+// words: 2 words of scratch (the max and the barrier's arrival count).
+qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *words,
                          cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s);
+    cudaError_t e = cudaMemsetAsync(words, 0, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
-    e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
-    if (e != cudaSuccess) return QT2_ERR_CUDA;
-    e = launch_fwd46_rows(static_cast<const uint16_t *>(x), rows, cols, ld, amax, out, s);
-    return from_cuda(e);
+    return from_cuda(launch_fwd46_coop(static_cast<const uint16_t *>(x), rows, cols, ld, words, out, s));
 }
 
 qt2_status gemm_enqueue(DevView a, DevView b, int64_t M, int64_t N, int64_t K, float alpha, void *c, int c_dtype,
@@ -397,7 +407,7 @@ DevView carve_view(Carve &c, int64_t R, int64_t C) {
 
 size_t linear_fwd_layout(int64_t M, int64_t K, int64_t N, void *ws, DevView *vx, DevView *vw, uint32_t **amax) {
     Carve c(ws);
-    *amax = reinterpret_cast<uint32_t *>(c.take(2 * sizeof(uint32_t)));
+    *amax = reinterpret_cast<uint32_t *>(c.take(4 * sizeof(uint32_t)));   // 2 words per quantizer call
     *vx = carve_view(c, M, K);
     *vw = carve_view(c, N, K);
     return c.used;
@@ -663,7 +673,7 @@ qt2_status qt2_linear_fwd(const void *x, const void *w, int64_t M, int64_t K, in
     if (st != QT2_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = fwd46_enqueue(x, M, K, K, vx, amax, s)) != QT2_OK) return st;
-    if ((st = fwd46_enqueue(w, N, K, K, vw, amax + 1, s)) != QT2_OK) return st;
+    if ((st = fwd46_enqueue(w, N, K, K, vw, amax + 2, s)) != QT2_OK) return st;
     return gemm_enqueue(vx, vw, M, N, K, 1.0f, y_bf16, QT2_DTYPE_BF16, N, s);
 }
 

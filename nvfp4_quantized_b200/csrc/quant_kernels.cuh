@@ -204,21 +204,78 @@ __device__ __forceinline__ float fwd46_tensor_scale(const uint32_t *amax_word) {
     return (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
 }
 
-__global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
-                                                         int64_t ld, const uint32_t *__restrict__ amax_word,
+// ---------------------------------------------------------------------------------------------
+// The forward quantizer in one cooperative launch: phase 1 merges max|x| of a grid-strided share
+// of the rows into words[0] (as amax_bf16_kernel); the CTAs meet at a grid barrier (arrivals
+// counted in words[1]; both words zeroed by the caller; every CTA is resident, which the
+// cooperative launch guarantees, and the wait is bounded); phase 2 quantizes exactly as
+// fwd46_group per 16-element group (one thread per group; four consecutive lanes hold the
+// four groups of one scale word).  A tensor that fits in L2 is read from HBM once.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(256) fwd46_coop_kernel(const uint16_t *__restrict__ x, int64_t R, int64_t C,
+                                                         int64_t ld, uint32_t *__restrict__ words,
                                                          uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
                                                          float *__restrict__ tensor_scale) {
-    const float g = fwd46_tensor_scale(amax_word);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    {   // phase 1: max |x| (bf16 magnitudes order like their bit patterns with the sign cleared)
+        const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+        const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+        const int64_t vec_per_row = C >> 3;
+        uint32_t m = 0;
+        for (int64_t r = gwarp; r < R; r += nwarps) {
+            const uint4 *row = reinterpret_cast<const uint4 *>(x + r * ld);
+#pragma unroll 4
+            for (int64_t v = lane; v < vec_per_row; v += 32) {
+                const uint4 w = row[v];
+                m = __vmaxu2(m, w.x & 0x7FFF7FFFu);
+                m = __vmaxu2(m, w.y & 0x7FFF7FFFu);
+                m = __vmaxu2(m, w.z & 0x7FFF7FFFu);
+                m = __vmaxu2(m, w.w & 0x7FFF7FFFu);
+            }
+        }
+        __shared__ uint32_t wmax[8];
+        const uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16) << 16);
+        if (lane == 0) wmax[warp] = bits;
+        __syncthreads();
+        __shared__ int gave_up;
+        if (threadIdx.x == 0) {
+            uint32_t b = 0;
+            for (int i = 0; i < 8; ++i) b = max(b, wmax[i]);
+            if (b) atomicMax(&words[0], b);
+            __threadfence();                                   // the max before the arrival
+            atomicAdd(&words[1], 1u);
+            int fail = 0;
+            const unsigned long long t0 = globaltimer_ns();
+            while (ld_acquire_gpu(&words[1]) < gridDim.x) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    set_device_error(QT2_ERR_TIMEOUT);
+                    fail = 1;
+                    break;
+                }
+                __nanosleep(100);
+            }
+            gave_up = fail;
+        }
+        __syncthreads();
+        if (gave_up) return;
+    }
+    // phase 2: the groups, one per thread and round, with the tensor's max
+    const float A = __uint_as_float(ld_acquire_gpu(&words[0]));
+    const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
     const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
     __shared__ float tab_d[128], tab_r[128];
     fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
-
-    const uint32_t G = (uint32_t)(C >> 4);                 // groups per row (a multiple of 8)
-    const uint64_t total = (uint64_t)R * G;                // a multiple of 1024
-    const bool small = total <= 0xFFFFFFFFull;              // 32-bit index arithmetic suffices
-    const int lane = threadIdx.x & 31;
+    const uint32_t G = (uint32_t)(C >> 4);
+    const uint64_t total = (uint64_t)R * G;
+    const bool small = total <= 0xFFFFFFFFull;
     for (uint64_t gi = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < total;
          gi += (uint64_t)gridDim.x * blockDim.x) {
         const uint64_t r = small ? (uint64_t)((uint32_t)gi / G) : gi / G;
@@ -229,7 +286,6 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
         uint32_t code0, code1;
         const uint32_t sc = fwd46_group(w, g6, g4, tab_d, tab_r, code0, code1);
         *reinterpret_cast<uint2 *>(codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8) = make_uint2(code0, code1);
-        // four consecutive groups (same row, q % 4 == 0 .. 3) share one scale word
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
@@ -242,7 +298,7 @@ __global__ void __launch_bounds__(256) fwd46_rows_kernel(const uint16_t *__restr
 // CTA-local forward quantizer ([FAF] "the speed-up is lost between the matmuls": the CTA-local
 // NVFP4 variant keeps the scale dependency inside a thread block; rows and columns get their own
 // corrections, constant over the summation and applied after it).  Block b of 128 rows is
-// quantized exactly as fwd46_rows_kernel does with the tensor scale g_b = A_b/1792 of its own
+// quantized exactly as fwd46_coop_kernel does, but with the tensor scale g_b = A_b/1792 of its own
 // max (1 below 2^-100) -- no grid-wide dependency, one launch.  A cluster of 4 CTAs owns a
 // block (32 rows each, so that 64-row weights still fill the GPU): each takes the max of its
 // rows, the four partial maxima meet through distributed shared memory, and each CTA then
