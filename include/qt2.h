@@ -95,7 +95,9 @@ QT2_API qt2_status qt2_device_status(qt2_stream_t stream, int *code);
  * layout_mask must be QT2_LAYOUT_ROW (the forward GEMM consumes row views only); row_out
  * receives the view (R = rows, C = cols); col_out is ignored and may be NULL.
  * One cooperative launch: its thread blocks merge the tensor max, meet at a grid barrier and
- * then quantize (a tensor that fits in L2 is read from HBM once).
+ * then quantize (a tensor that fits in L2 is read from HBM once).  Work kept running by other
+ * streams on the same GPU can delay the barrier; after 2 s the call gives up, quantizes nothing
+ * and reports QT2_ERR_TIMEOUT through qt2_device_status.
  * Workspace: at least qt2_quant_fwd46_workspace_size() bytes, 16-byte aligned; it holds the
  * tensor max and the barrier's counter and is overwritten.
  * --------------------------------------------------------------------------------------- */
