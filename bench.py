@@ -136,6 +136,28 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------- our arm
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank passes its own device-timed milliseconds and gets the
+    maximum back (one all-reduce; a single rank returns its own)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own batch (weak scaling), so the
+    job does world * steps * flops in the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def rank_input_seed(rank: int, set_index: int) -> int:
+    """Seed of input set `set_index` (two alternate) on `rank`: each rank draws its own batch."""
+    return 1000 * rank + 10 * set_index
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -151,7 +173,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # two resident input sets (seeded per rank), outputs and every intermediate view
     sets = []
     for i in range(2):
-        x, w, dy = synth.linear_inputs(args.config, seed=1000 * rank + 10 * i, device=dev)
+        x, w, dy = synth.linear_inputs(args.config, seed=rank_input_seed(rank, i), device=dev)
         sets.append((x, w, dy))
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
@@ -283,10 +305,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     status = Q.qt2_device_status(stream)
     per = {n: sum(events[i][j].elapsed_time(events[i][j + 1]) for i in range(args.steps)) / args.steps
            for j, n in enumerate(names)}
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # ------------------------------------------------------------------ end to end through the API
     # Every step uploads X, W, dY from pinned host memory, runs qt2_linear_fwd + qt2_linear_bwd and
@@ -357,14 +376,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         s_in.wait_stream(s_out)
         e_e.record(s_in)
         torch.cuda.synchronize()
-        te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te_ms = max_over_ranks(e_s.elapsed_time(e_e), world, dev)
         flops_step = 3 * 2.0 * M * N * K
-        e2e = {"value": world * flops_step * n_e2e / (float(te.item()) * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_tflops(world, flops_step, n_e2e, te_ms), "unit": UNIT,
                "h2d_bytes_per_step": hx.numel() * 2 + hw.numel() * 2 + hdy.numel() * 2,
                "d2h_bytes_per_step": hy.numel() * 2 + hdx.numel() * 2 + hdw.numel() * 4,
-               "steps": n_e2e, "ms_per_step": float(te.item()) / n_e2e,
+               "steps": n_e2e, "ms_per_step": te_ms / n_e2e,
                "pipeline": "3 streams (upload, compute, download), 2 device buffer sets"}
     return dict(M=M, K=K, N=N, max_ms=max_ms, per=per, status=status, clocks=clk.summary(), e2e=e2e)
 
@@ -489,7 +506,7 @@ def main():
     pk = peaks()
     flops_gemm = 2.0 * M * N * K
     flops_step = 3 * flops_gemm
-    value = world * flops_step * args.steps / (r["max_ms"] * 1e-3) / 1e12
+    value = job_tflops(world, flops_step, args.steps, r["max_ms"])
     per = r["per"]
     gemm_ms = (per["gemm_fwd"] + per["gemm_dgrad"] + per["gemm_wgrad"]) / 3
     fp4_peak = pk["bf16_sustained"] * 4.0
