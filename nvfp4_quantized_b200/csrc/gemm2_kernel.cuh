@@ -132,12 +132,6 @@ __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&p)[8]) 
                  : "memory");
 }
 
-// One lane of a converged warp (PTX elect.sync).
-__device__ __forceinline__ bool elect_one() {
-    uint32_t p;
-    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xFFFFFFFF;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(p));
-    return p != 0;
-}
 
 // ------------------------------------------------------------------ configuration
 struct Gemm2Cfg {

@@ -8,16 +8,19 @@
 // with both operands K-major ("TN"), 1x16 E4M3 scales, fp32 accumulation in tensor memory.
 //
 // Design (one CTA of 128 threads per 128 x BN output tile):
-//   warp 0, one thread : producer -- TMA loads of the A/B code tiles (128-byte swizzle, no
+//   warp 0             : producer -- TMA loads of the A/B code tiles (128-byte swizzle, no
 //                        multicast) and bulk copies of the 512-byte scale atoms into a ring of
 //                        STAGES shared-memory stages, each covering K = 256.
-//   warp 1, one thread : MMA issuer -- per stage, tcgen05.cp of the scale atoms into TMEM
+//   warp 1             : MMA issuer -- per stage, tcgen05.cp of the scale atoms into TMEM
 //                        (replicated into the four lane quadrants), then four
 //                        tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 each); tcgen05.commit
 //                        frees the stage once those MMAs have completed.
 //   warp 2             : allocates and frees the TMEM columns.
 //   all four warps     : epilogue -- tcgen05.ld of the fp32 accumulator (warp w owns lanes
 //                        32w..32w+31 = tile rows), scale by alpha*gA*gB, store bf16 or fp32.
+// Warps 0 and 1 run converged and let one lane chosen by elect.sync issue (TMA, bulk copies and
+// tcgen05 instructions take warp-uniform operands; issued from a lone lane of a diverged warp
+// each pays extra issue work).
 // Every wait is bounded (mbar_wait); a timeout records QT2_ERR_TIMEOUT and the CTA still
 // reaches the common exit, frees its TMEM and returns.
 #pragma once
@@ -91,50 +94,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t t_acc = tmem, t_sfa = tmem + BN, t_sfb = tmem + BN + 16;
 
-    if (warp == 0 && lane == 0) {
-        // ---------------------------------------------------------------- producer
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer (whole warp,
+        // one elected lane issues: TMA and bulk copies take warp-uniform operands)
         const uint8_t *sfa_blk = sfa + (m0 >> 7) * (int64_t)nkb * 512;
         for (int ks = 0; ks < nks; ++ks) {
             const int s = ks % S;
-            if (ks >= S && !mbar_wait(empty0 + 8 * s, ((ks / S) & 1) ^ 1)) break;
+            if (ks >= S && !mbar_wait_warp(empty0 + 8 * s, ((ks / S) & 1) ^ 1)) break;
             const int kb0 = ks * 4, nk = min(4, nkb - kb0);
             const uint32_t fb = full0 + 8 * s;
-            mbar_arrive_expect_tx(fb, Cfg::kABytes + Cfg::kBBytes + nk * 512 * (1 + BN / 128));
-            tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmA, ks * kGemmBKBytes, (int32_t)m0, fb);
-            tma_load_2d(smem_u32(sB + s * Cfg::kBBytes), &tmB, ks * kGemmBKBytes, (int32_t)n0, fb);
-            bulk_load(smem_u32(sSFA + s * Cfg::kSfaBytes), sfa_blk + (int64_t)kb0 * 512, nk * 512, fb);
+            if (elect_one()) {
+                mbar_arrive_expect_tx(fb, Cfg::kABytes + Cfg::kBBytes + nk * 512 * (1 + BN / 128));
+                tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmA, ks * kGemmBKBytes, (int32_t)m0, fb);
+                tma_load_2d(smem_u32(sB + s * Cfg::kBBytes), &tmB, ks * kGemmBKBytes, (int32_t)n0, fb);
+                bulk_load(smem_u32(sSFA + s * Cfg::kSfaBytes), sfa_blk + (int64_t)kb0 * 512, nk * 512, fb);
 #pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
-                bulk_load(smem_u32(sSFB + s * Cfg::kSfbBytes + h * 2048),
-                          sfb + (((n0 >> 7) + h) * (int64_t)nkb + kb0) * 512, nk * 512, fb);
+                for (int h = 0; h < BN / 128; ++h)
+                    bulk_load(smem_u32(sSFB + s * Cfg::kSfbBytes + h * 2048),
+                              sfb + (((n0 >> 7) + h) * (int64_t)nkb + kb0) * 512, nk * 512, fb);
+            }
+            __syncwarp();
             issued = ks + 1;
         }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------------------------------------------------------- MMA issuer
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer (whole warp,
+        // one elected lane issues)
         for (int ks = 0; ks < nks; ++ks) {
             const int s = ks % S;
-            if (!mbar_wait(full0 + 8 * s, (ks / S) & 1)) break;
-            *consumed_slot = ks + 1;
+            if (!mbar_wait_warp(full0 + 8 * s, (ks / S) & 1)) break;
+            if (lane == 0) *consumed_slot = ks + 1;
             tc_fence_after();
             const int nk = min(4, nkb - ks * 4);
             const uint32_t a_s = smem_u32(sA + s * Cfg::kABytes), b_s = smem_u32(sB + s * Cfg::kBBytes);
             const uint32_t sfa_s = smem_u32(sSFA + s * Cfg::kSfaBytes), sfb_s = smem_u32(sSFB + s * Cfg::kSfbBytes);
-            for (int kk = 0; kk < nk; ++kk) {
-                tc_cp_32x128b_warpx4(t_sfa + 4 * kk, make_smem_desc(sfa_s + 512 * kk, 0, 128, 0));
+            if (elect_one()) {
+                for (int kk = 0; kk < nk; ++kk) {
+                    tc_cp_32x128b_warpx4(t_sfa + 4 * kk, make_smem_desc(sfa_s + 512 * kk, 0, 128, 0));
 #pragma unroll
-                for (int h = 0; h < BN / 128; ++h)
-                    tc_cp_32x128b_warpx4(t_sfb + (BN / 32) * kk + 4 * h,
-                                         make_smem_desc(sfb_s + 2048 * h + 512 * kk, 0, 128, 0));
+                    for (int h = 0; h < BN / 128; ++h)
+                        tc_cp_32x128b_warpx4(t_sfb + (BN / 32) * kk + 4 * h,
+                                             make_smem_desc(sfb_s + 2048 * h + 512 * kk, 0, 128, 0));
+                }
+                for (int kk = 0; kk < nk; ++kk) {
+                    const uint64_t adesc = make_smem_desc(a_s + 32 * kk, 16, 1024, 2);
+                    const uint64_t bdesc = make_smem_desc(b_s + 32 * kk, 16, 1024, 2);
+                    tc_mma_nvfp4(t_acc, adesc, bdesc, Cfg::kIdesc, t_sfa + 4 * kk, t_sfb + (BN / 32) * kk,
+                                 (ks | kk) != 0);
+                }
+                tc_commit(empty0 + 8 * s);
             }
-            for (int kk = 0; kk < nk; ++kk) {
-                const uint64_t adesc = make_smem_desc(a_s + 32 * kk, 16, 1024, 2);
-                const uint64_t bdesc = make_smem_desc(b_s + 32 * kk, 16, 1024, 2);
-                tc_mma_nvfp4(t_acc, adesc, bdesc, Cfg::kIdesc, t_sfa + 4 * kk, t_sfb + (BN / 32) * kk,
-                             (ks | kk) != 0);
-            }
-            tc_commit(empty0 + 8 * s);
+            __syncwarp();
         }
-        tc_commit(accum_bar);
+        if (elect_one()) tc_commit(accum_bar);
     }
     __syncwarp();
 
