@@ -18,6 +18,15 @@ the max over ranks and value = all ranks' FLOPs / that time.
 
 --impl reference times the CPU oracle (the plain restatement the CUDA path is checked
 against) on a bounded sample of the same workload, on the host cores, rank 0 only.
+
+Other lines (same JSON contract):
+  --schedule fused   X's forward and MS-EDEN column views from one read; W's two views made
+                     once before the timed steps (micro-batches of one optimizer step).
+  --schedule local   the forward with CTA-local (per-128-row-block) tensor scales.
+  --op fwd46_sq      the 16x16 square-block weight quantizer alone, on W of the config.
+  --config mlp8b_up | mlp8b_down   the Llama-3-8B MLP linears at 16384 tokens.
+The end-to-end leg (`e2e`) runs qt2_linear_fwd + qt2_linear_bwd with every input uploaded from
+pinned host memory and every output downloaded each step, pipelined over three streams.
 """
 from __future__ import annotations
 
