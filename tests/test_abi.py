@@ -69,6 +69,9 @@ def test_host_validation_codes(L):
     R = ctypes.byref
     assert f(None, 128, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_INVALID_ARG
     assert f(0x1000, 100, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
+    assert f(0x1000, 0, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE      # empty
+    assert f(0x1000, 128, 0, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
+    assert f(0x1000, -128, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
     assert f(0x1000, 128, 128, 64, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_SHAPE
     assert f(0x1008, 128, 128, 128, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
     assert f(0x1000, 128, 128, 132, 1, R(v), None, 0x40000, 256, None) == qt2.QT2_ERR_ALIGN
@@ -85,6 +88,8 @@ def test_host_validation_codes(L):
     assert h(R(v), R(v), 128, 128, 128, 1.0, 0x50000, 7, 128, None) == qt2.QT2_ERR_INVALID_ARG
     assert h(R(v), R(v), 128, 192, 128, 1.0, 0x50000, 0, 192, None) == qt2.QT2_ERR_SHAPE
     assert h(R(v), R(v), 128, 128, 128, 1.0, 0x50000, 0, 64, None) == qt2.QT2_ERR_SHAPE
+    assert h(R(v), R(v), 128, 128, 0, 1.0, 0x50000, 0, 128, None) == qt2.QT2_ERR_SHAPE       # empty K
+    assert h(R(v), R(v), 0, 128, 128, 1.0, 0x50000, 0, 128, None) == qt2.QT2_ERR_SHAPE
     assert L.qt2_linear_fwd(0x1000, 0x2000, 128, 128, 128, 0x3000, None, 0, None) == qt2.QT2_ERR_WORKSPACE
     assert L.qt2_linear_bwd(0x1000, 0x2000, 0x3000, 128, 128, 128, 0, 0x4000, 0x5000, 3, 0x6000, 1 << 30,
                             None) == qt2.QT2_ERR_INVALID_ARG
