@@ -1,4 +1,8 @@
-// quant_kernels.cuh -- the HBM-bound producers of the NVFP4 views (sm_100a).
+// quant_kernels.cuh -- the forward quantizers and MS-EDEN's scale pass (sm_100a): the tensor max,
+// the forward quantizer in one cooperative launch (fwd46_coop_kernel), its CTA-local
+// (fwd46_local_kernel) and 16x16 square-block (fwd46_sq_kernel) variants, and the MS-EDEN
+// finalize (msed_finalize_kernel).  They read and write HBM streams but are bound by their
+// per-element arithmetic, which follows the reference order exactly.
 //
 // Citations (page title, then section):
 //   [QII-th] "Quartet II ... MS-EDEN" Thai translation (itsolotime.com archives 22992): "Question 1"
