@@ -280,6 +280,14 @@ QT2_API qt2_status qt2_linear_bwd_views(const void *dy, int64_t M, int64_t K, in
                                         void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
                                         qt2_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Self-test of the device error path: enqueues one kernel whose single wait (on a barrier that
+ * nothing completes) gives up after the library's wait limit (2 s) and records QT2_ERR_TIMEOUT
+ * in the device status word, exactly as a real wait would; qt2_device_status then returns it
+ * (and clears it).  Nothing else is touched; the context stays usable.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

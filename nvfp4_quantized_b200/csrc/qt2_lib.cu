@@ -64,6 +64,18 @@ cudaError_t launch_fwd46_coop(const uint16_t *x, int64_t R, int64_t C, int64_t l
     return cudaLaunchCooperativeKernel((const void *)fwd46_coop_kernel, dim3((unsigned)blocks), dim3(256), args, 0, s);
 }
 
+// Self-test of the error path of a device wait: one thread waits on an mbarrier that nothing
+// arrives at; the bounded wait gives up after kWaitLimitNs and records QT2_ERR_TIMEOUT.
+__global__ void selftest_wait_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0);
+}
+
 cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t ld, DevView out, cudaStream_t s) {
     fwd46_local_kernel<<<(unsigned)(R / 128 * kLocalCluster), kLocalThreads, 0, s>>>(x, R, C, ld, out.codes,
                                                                                      out.scales, out.tensor_scale);
@@ -715,6 +727,13 @@ qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t 
     if ((st = gemm_enqueue(L.dy_row, L.w_col, M, K, N, 0x1p-7f, dx_bf16, QT2_DTYPE_BF16, K, s)) != QT2_OK) return st;
     // wgrad: dW[N][K] = 2^-7 * dY_col[N][M] . X_col[K][M]^T
     return gemm_enqueue(L.dy_col, L.x_col, N, K, M, 0x1p-7f, dw, dw_dtype, K, s);
+}
+
+qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream) {
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return from_cuda(cudaGetLastError());
 }
 
 qt2_status qt2_quant_fwd46_local(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,

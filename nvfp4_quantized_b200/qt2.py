@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
                 "qt2_linear_bwd_workspace_size": (i32, [i64, i64, i64, psz]),
                 "qt2_linear_bwd": (i32, [vp, vp, vp, i64, i64, i64, u64, vp, vp, i32, vp, sz, vp]),
                 "qt2_quant_fwd46_local": (i32, [vp, i64, i64, i64, pv, vp]),
+                "qt2_selftest_wait_timeout": (i32, [vp]),
                 "qt2_gemm_nvfp4_local": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
@@ -320,3 +321,8 @@ def qt2_gemm_nvfp4_local(a: View, b: View, M: int, N: int, K: int, alpha: float,
     ac, bc = a.c(), b.c()
     _check("qt2_gemm_nvfp4_local", lib().qt2_gemm_nvfp4_local(ctypes.byref(ac), ctypes.byref(bc), M, N, K, alpha,
                                                               _ptr(c), c_dtype, ldc, _stream(stream)))
+
+
+def qt2_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the device wait self-test (its wait gives up after the library's limit)."""
+    _check("qt2_selftest_wait_timeout", lib().qt2_selftest_wait_timeout(_stream(stream)))

@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 23
+    assert len(names) == 24
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -129,6 +129,7 @@ def test_valid_call_without_gpu_fails_loudly(L):
     v = _view()
     st = L.qt2_quant_fwd46(0x1000, 128, 128, 128, 1, ctypes.byref(v), None, 0x40000, 256, None)
     assert st == qt2.QT2_ERR_DEVICE
+    assert L.qt2_selftest_wait_timeout(None) == qt2.QT2_ERR_DEVICE
     with pytest.raises(qt2.QT2Error):
         qt2._check("qt2_quant_fwd46", st)
 
