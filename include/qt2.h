@@ -21,6 +21,12 @@
  *     ld >= cols, ld a multiple of 8) and 16-byte aligned base pointers.
  *   - Every dimension must be a positive multiple of 128.
  *   - The device must be compute capability 10.0 (B200); otherwise QT2_ERR_DEVICE.
+ *   - Inputs must be finite.  A quantizer that meets inf or NaN in its input records
+ *     QT2_ERR_NONFINITE in the device status word (qt2_device_status); what its outputs then
+ *     hold is unspecified.  The rotating quantizers (MS-EDEN, SR) report the same when the
+ *     rotation overflows binary32 (a block sum of 128 inputs beyond 3.4e38, i.e. |x| above
+ *     about 2^121).  The method is defined on real numbers only.
+ *   - One NVTX range per call, named after the call, marks it for profilers.
  *
  * NVFP4 view layout (one quantized operand of a "TN" GEMM, grouped along its contraction axis):
  *   R = rows (non-contraction axis), C = columns (contraction axis), both multiples of 128.
@@ -58,7 +64,8 @@ typedef enum {
     QT2_ERR_WORKSPACE = -4,   /* workspace null or smaller than the size query returned */
     QT2_ERR_CUDA = -5,        /* a CUDA runtime/driver call or launch failed */
     QT2_ERR_TIMEOUT = -6,     /* a device-side bounded wait gave up (see qt2_device_status) */
-    QT2_ERR_DEVICE = -7       /* no device, or the current device is not sm_100 */
+    QT2_ERR_DEVICE = -7,      /* no device, or the current device is not sm_100 */
+    QT2_ERR_NONFINITE = -8    /* device-side: an input held inf or NaN (see qt2_device_status) */
 } qt2_status;
 
 enum { QT2_LAYOUT_ROW = 1, QT2_LAYOUT_COL = 2, QT2_LAYOUT_BOTH = 3 };
@@ -77,9 +84,21 @@ QT2_API int qt2_version(void);
 QT2_API const char *qt2_status_string(qt2_status s);
 
 /* Reads and clears the library's device-side status word after synchronizing `stream`.
- * *code = 0 when no kernel reported a problem; QT2_ERR_TIMEOUT when a bounded wait gave up.
+ * *code = 0 when no kernel reported a problem; QT2_ERR_TIMEOUT when a bounded wait gave up;
+ * QT2_ERR_NONFINITE when a quantizer met inf or NaN in its input (the first report wins).
  * Synchronizes the stream; meant for tests and debugging, not the hot path. */
 QT2_API qt2_status qt2_device_status(qt2_stream_t stream, int *code);
+
+/* Host-side fault injection, for testing callers' error handling without a GPU fault.
+ * While a hook is set, every CUDA call the library makes while enqueuing work is first
+ * announced as hook(site, user), site one of "device" (the device query), "tensor_map" (a TMA
+ * descriptor), "memset", "launch" and "symbol" (the scratch lookup of qt2_quant_msedEN_noalloc).  The hook returns 0 to let the call happen, 1 to make it
+ * fail without being made (the entry point then returns QT2_ERR_DEVICE for "device" and
+ * QT2_ERR_CUDA otherwise, having enqueued nothing further), or 2 to skip it and report success
+ * (so a test can walk past the device query on a machine without a GPU).  NULL removes the
+ * hook.  Meant for tests: set it while no other thread is calling into the library. */
+typedef int (*qt2_fault_hook)(const char *site, void *user);
+QT2_API void qt2_set_fault_hook(qt2_fault_hook hook, void *user);
 
 /* ---------------------------------------------------------------------------------------
  * Forward quantizer: round-to-nearest onto E2M1 in 1x16 groups with the "4/6" grid choice.
@@ -200,13 +219,15 @@ QT2_API qt2_status qt2_quant_sr(const void *x_bf16, int64_t rows, int64_t cols, 
  * must not call cudaMalloc, a plugin whose host framework owns the allocator).
  *
  * Same arguments and results as qt2_quant_msedEN (bit-identical outputs), minus the
- * workspace: the scratch lives in a fixed device array of QT2_NOALLOC_SCRATCH_BYTES (32 MiB)
- * inside the library, which every GPU that loads the library holds until the process exits.
- * A call needs 256 bytes plus rows*cols/4 bytes per requested view, so at most about 64 Mi
- * elements with QT2_LAYOUT_BOTH or 128 Mi elements with one view (for example 8192 x 8192
- * both views); larger tensors return QT2_ERR_WORKSPACE and enqueue nothing.
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.
+ * workspace: the scratch lives in a fixed device array inside the library -- a 256-byte slot
+ * for the two view maxima plus QT2_NOALLOC_SCRATCH_BYTES (32 MiB) for the fp32 pre-scales --
+ * which every GPU that loads the library holds until the process exits.  The pre-scales take
+ * rows*cols/4 bytes per requested view, so the call accepts up to 64 Mi elements with
+ * QT2_LAYOUT_BOTH (for example 8192 x 8192) and up to 128 Mi elements with one view (for
+ * example 8192 x 16384); larger tensors return QT2_ERR_WORKSPACE and enqueue nothing.
+ * Every call looks up the array's device address (cudaGetSymbolAddress) with the calling
+ * device current, so the address stays right after a device reset.  The first call on a device
+ * may load the library's device code there; make it before any stream capture.
  * All calls on a device share the one array: the call zeroes the view maxima it needs and
  * rewrites every pre-scale before reading it, but two calls whose work overlaps on the GPU
  * (different streams without ordering between them) race on the array and give wrong results.

@@ -69,15 +69,22 @@ __device__ __forceinline__ float div6_rn(float a) {
     return __fmaf_rn(rem, kSixth, q0);
 }
 
-// max(|a|, |b|, |c|) (sm_100a three-input max; exact, so the grouping does not matter)
+// max(|a|, |b|, |c|) (sm_100a three-input max; exact, so the grouping does not matter).  The
+// .NaN forms return NaN when an operand is NaN, so a non-finite input reaches the view max
+// (y holds inf or NaN wherever a block of x held one) and is reported by the scale pass.
 __device__ __forceinline__ float absmax3(float a, float b, float c) {
     float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
     return r;
 }
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float max2n(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
     return r;
 }
 
@@ -154,8 +161,8 @@ __device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint
         const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
         const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
         const float m4 = absmax3(y[12], y[13], y[14]);
-        const float a = fmaxf(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
-        amax = fmaxf(amax, a);
+        const float a = max2n(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+        amax = max2n(amax, a);
         const bool live = a >= kTiny;
         const float p = live ? div6_rn(a) : 0.0f;
         const float r = live ? __frcp_rn(p) : 0.0f;          // flushed group: sign-preserving zeros
@@ -229,8 +236,8 @@ __device__ __forceinline__ void sr_vector(const uint64_t (&P)[32], float g, floa
         const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
         const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
         const float m4 = absmax3(y[12], y[13], y[14]);
-        const float a = fmaxf(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
-        amax = fmaxf(amax, a);
+        const float a = max2n(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+        amax = max2n(amax, a);
         float q[16];
         if (zero_view || !(a >= kTiny)) {
             sc[gq] = 0;
@@ -362,6 +369,10 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     float g_r = 1.0f, g6_r = 6.0f, g_c = 1.0f, g6_c = 6.0f;
     bool zero_r = true, zero_c = true;
     if constexpr (MODE == kModeSr) {
+        if (blockIdx.x == 0 && t == 0) {
+            if (DO_ROW) check_finite_word(*row_amax);
+            if (DO_COL) check_finite_word(*col_amax);
+        }
         if (DO_ROW) {
             const float A = __uint_as_float(*row_amax);
             zero_r = !(A >= kTiny);
@@ -381,6 +392,7 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     __shared__ float tab_d[128], tab_r[128];
     float g6_f = 0.0f, g4_f = 0.0f;
     if constexpr (MODE == kModeFwdRowEdenCol) {
+        if (blockIdx.x == 0 && t == 0) check_finite_word(*row_amax);   // outputs then unspecified
         const float g = fwd46_tensor_scale(row_amax);
         g6_f = __fmul_rn(g, 6.0f);
         g4_f = __fmul_rn(g, 4.0f);

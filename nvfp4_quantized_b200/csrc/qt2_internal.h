@@ -6,6 +6,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "qt2.h"
 
@@ -46,6 +47,24 @@ cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tm
 // 2D tensor map for TMA (no multicast anywhere in this library).
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+// Host-side fault injection (qt2_set_fault_hook).  Every CUDA call the library makes while
+// enqueuing passes through fault_at(site) first: kFaultNone = make the call, kFaultFail = report
+// the call as failed without making it, kFaultSkip = report success without making it.
+enum FaultAction { kFaultNone = 0, kFaultFail = 1, kFaultSkip = 2 };
+int fault_at(const char *site);
+
+// One NVTX range per C call, named after the call (free unless a profiler is attached).
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+};
+#define QT2_TRACE() ::qt2::TraceRange qt2_trace_range_(__func__)
+
+// Device ordinal of the calling thread (-1 when there is none).  Attribute and occupancy caches
+// are kept per device, for the first kMaxDevices devices.
+constexpr int kMaxDevices = 64;
+int current_device();
 
 // Hooks used by the workspace-free MS-EDEN entry point (qt2_noalloc.cu).
 qt2_status msed_check_args(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,

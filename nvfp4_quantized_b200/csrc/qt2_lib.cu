@@ -21,23 +21,80 @@
 namespace qt2 {
 
 // ---------------------------------------------------------------------------------------------
+// host-side fault injection and per-device caches
+// ---------------------------------------------------------------------------------------------
+static std::atomic<qt2_fault_hook> g_fault_hook{nullptr};
+static std::atomic<void *> g_fault_user{nullptr};
+
+int fault_at(const char *site) {
+    const qt2_fault_hook h = g_fault_hook.load(std::memory_order_acquire);
+    if (h == nullptr) return kFaultNone;
+    const int a = h(site, g_fault_user.load(std::memory_order_acquire));
+    return (a == kFaultFail || a == kFaultSkip) ? a : kFaultNone;
+}
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return dev;
+}
+
+// One-time set-up per device (function attributes, occupancy): f() runs with the device
+// current until it has succeeded once there.  A process that drives several GPUs sets every
+// kernel up on each of them.
+struct PerDeviceOnce {
+    std::atomic<int> done[kMaxDevices];
+    template <class F>
+    cudaError_t run(F &&f) {
+        const int dev = current_device();
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        const cudaError_t e = f();
+        if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+        return e;
+    }
+};
+
+// Launch sites consult the fault hook: a failure is reported as a failed launch, a skip as a
+// successful one, and in both cases nothing is launched.
+#define QT2_LAUNCH_SITE()                                        \
+    do {                                                         \
+        const int fa_ = fault_at("launch");                      \
+        if (fa_ == kFaultFail) return cudaErrorLaunchFailure;    \
+        if (fa_ == kFaultSkip) return cudaSuccess;               \
+    } while (0)
+
+static cudaError_t memset_async(void *p, size_t n, cudaStream_t s) {
+    const int fa = fault_at("memset");
+    if (fa == kFaultFail) return cudaErrorInvalidValue;
+    if (fa == kFaultSkip) return cudaSuccess;
+    return cudaMemsetAsync(p, 0, n, s);
+}
+
+// ---------------------------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------------------------
 static int sm_count() {
-    static std::atomic<int> cached{0};
-    int v = cached.load();
+    static std::atomic<int> cached[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int v = cached[dev].load();
     if (v == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        if (v <= 0) v = 148;
-        cached.store(v);
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            cudaGetLastError();
+            v = 148;
+        }
+        cached[dev].store(v);
     }
     return v;
 }
 
 cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *amax_word,
                              cudaStream_t s) {
+    QT2_LAUNCH_SITE();
     const int64_t warps_needed = R;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((warps_needed + 7) / 8, (int64_t)sm_count() * 8));
     amax_bf16_kernel<<<blocks, 256, 0, s>>>(x, R, C, ld, amax_word);
@@ -49,11 +106,17 @@ cudaError_t launch_amax_bf16(const uint16_t *x, int64_t R, int64_t C, int64_t ld
 // barrier's arrivals).  The grid is every CTA that fits on the device at once.
 cudaError_t launch_fwd46_coop(const uint16_t *x, int64_t R, int64_t C, int64_t ld, uint32_t *words, DevView out,
                               cudaStream_t s) {
-    static std::once_flag once;
-    static int per_sm = 0;
-    static cudaError_t occ_err = cudaSuccess;
-    std::call_once(once, [] { occ_err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd46_coop_kernel, 256, 0); });
+    QT2_LAUNCH_SITE();
+    static PerDeviceOnce once;
+    static std::atomic<int> occupancy[kMaxDevices];
+    const cudaError_t occ_err = once.run([] {
+        int v = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fwd46_coop_kernel, 256, 0);
+        if (e == cudaSuccess) occupancy[current_device()].store(v);
+        return e;
+    });
     if (occ_err != cudaSuccess) return occ_err;
+    const int per_sm = occupancy[current_device()].load();
     if (per_sm < 1) return cudaErrorLaunchOutOfResources;
     const int64_t groups = R * (C >> 4);
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((groups + 255) / 256, (int64_t)per_sm * sm_count()));
@@ -77,6 +140,7 @@ __global__ void selftest_wait_kernel() {
 }
 
 cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t ld, DevView out, cudaStream_t s) {
+    QT2_LAUNCH_SITE();
     fwd46_local_kernel<<<(unsigned)(R / 128 * kLocalCluster), kLocalThreads, 0, s>>>(x, R, C, ld, out.codes,
                                                                                      out.scales, out.tensor_scale);
     return cudaGetLastError();
@@ -84,6 +148,7 @@ cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t 
 
 cudaError_t launch_fwd46_sq(const uint16_t *x, int64_t R, int64_t C, int64_t ld, const uint32_t *amax_word,
                             DevView row, DevView col, cudaStream_t s) {
+    QT2_LAUNCH_SITE();
     const int64_t pairs = (R / 16) * (C / 16) / 2;   // two 16x16 blocks per warp
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((pairs + 7) / 8, (int64_t)sm_count() * 16));
     fwd46_sq_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, R, C, ld, amax_word, row.codes, row.scales, row.tensor_scale,
@@ -94,11 +159,11 @@ cudaError_t launch_fwd46_sq(const uint16_t *x, int64_t R, int64_t C, int64_t ld,
 template <int MODE, bool ROW, bool COL>
 static cudaError_t launch_rot_variant(const CUtensorMap &tmap, int64_t R, int64_t C, uint64_t seed,
                                       const RotViews &out, cudaStream_t s) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(msed_kernel<MODE, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        MsedCfg::kSmemBytes);
+    QT2_LAUNCH_SITE();
+    static PerDeviceOnce once;
+    const cudaError_t attr_err = once.run([] {
+        return cudaFuncSetAttribute(msed_kernel<MODE, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    MsedCfg::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     const int64_t ntiles = (R >> 7) * (C >> 7);
@@ -158,6 +223,7 @@ static FinalizeJob finalize_job(const float *P, int64_t R, int64_t C, const uint
 cudaError_t launch_msed_finalize(const float *P_a, int64_t R_a, int64_t C_a, const uint32_t *amax_a, uint32_t tid_a,
                                  DevView out_a, const float *P_b, int64_t R_b, int64_t C_b, const uint32_t *amax_b,
                                  uint32_t tid_b, DevView out_b, uint64_t seed, cudaStream_t s) {
+    QT2_LAUNCH_SITE();
     const int64_t cap = (int64_t)sm_count() * 16;
     FinalizeJob ja = finalize_job(P_a, R_a, C_a, amax_a, tid_a, out_a, P_b ? cap / 2 : cap);
     FinalizeJob jb = P_b ? finalize_job(P_b, R_b, C_b, amax_b, tid_b, out_b, cap / 2) : ja;
@@ -170,11 +236,11 @@ template <int BN>
 static cudaError_t launch_gemm_bn(const CUtensorMap &tmA, const CUtensorMap &tmB, DevView a, DevView b, int64_t M,
                                   int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
                                   cudaStream_t s, int local) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        GemmCfg<BN>::kSmemBytes);
+    QT2_LAUNCH_SITE();
+    static PerDeviceOnce once;
+    const cudaError_t attr_err = once.run([] {
+        return cudaFuncSetAttribute(gemm_nvfp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    GemmCfg<BN>::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     dim3 grid((unsigned)(N / BN), (unsigned)(M / kGemmBM));
@@ -194,11 +260,11 @@ cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tm
                                    const CUtensorMap &tmSFB, DevView a, DevView b, int64_t M,
                                    int64_t N, int64_t K, float alpha, void *c, int c_dtype, int64_t ldc,
                                    cudaStream_t s, int local) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        Gemm2Cfg::kSmemBytes);
+    QT2_LAUNCH_SITE();
+    static PerDeviceOnce once;
+    const cudaError_t attr_err = once.run([] {
+        return cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Gemm2Cfg::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     const int64_t tiles = (M / 256) * (N / 256);
@@ -231,6 +297,12 @@ static EncodeTiledFn encode_fn() {
 
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    const int fa = fault_at("tensor_map");
+    if (fa == kFaultFail) return false;
+    if (fa == kFaultSkip) {
+        std::memset(map, 0, sizeof(*map));
+        return true;
+    }
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -260,6 +332,9 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool dim_ok(int64_t d) { return d > 0 && d % 128 == 0 && d <= (int64_t(1) << 31); }
 
 qt2_status check_device() {
+    const int fa = fault_at("device");
+    if (fa == kFaultFail) return QT2_ERR_DEVICE;
+    if (fa == kFaultSkip) return QT2_OK;
     static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
@@ -329,7 +404,7 @@ qt2_status msed_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, i
     if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
                         128, CU_TENSOR_MAP_SWIZZLE_128B))
         return QT2_ERR_CUDA;
-    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    cudaError_t e = memset_async(amax, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     e = launch_msed_tiles(tmap, rows, cols, (mask & QT2_LAYOUT_ROW) != 0, (mask & QT2_LAYOUT_COL) != 0, seed, row, col,
                           P_row, P_col, amax, amax + 1, s);
@@ -353,7 +428,7 @@ qt2_status fwd46_msed_col_enqueue(const void *x, int64_t rows, int64_t cols, int
     if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
                         128, CU_TENSOR_MAP_SWIZZLE_128B))
         return QT2_ERR_CUDA;
-    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    cudaError_t e = memset_async(amax, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
@@ -365,7 +440,7 @@ qt2_status fwd46_msed_col_enqueue(const void *x, int64_t rows, int64_t cols, int
 
 qt2_status fwd46_sq_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView row, DevView col,
                             uint32_t *amax, cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(uint32_t), s);
+    cudaError_t e = memset_async(amax, sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     e = launch_amax_bf16(static_cast<const uint16_t *>(x), rows, cols, ld, amax, s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
@@ -376,7 +451,7 @@ qt2_status fwd46_sq_enqueue(const void *x, int64_t rows, int64_t cols, int64_t l
 // words: 2 words of scratch (the max and the barrier's arrival count).
 qt2_status fwd46_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, DevView out, uint32_t *words,
                          cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(words, 0, 2 * sizeof(uint32_t), s);
+    cudaError_t e = memset_async(words, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     return from_cuda(launch_fwd46_coop(static_cast<const uint16_t *>(x), rows, cols, ld, words, out, s));
 }
@@ -499,7 +574,7 @@ qt2_status sr_enqueue(const void *x, int64_t rows, int64_t cols, int64_t ld, int
     if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64,
                         128, CU_TENSOR_MAP_SWIZZLE_128B))
         return QT2_ERR_CUDA;
-    cudaError_t e = cudaMemsetAsync(amax, 0, 2 * sizeof(uint32_t), s);
+    cudaError_t e = memset_async(amax, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess) return QT2_ERR_CUDA;
     const bool do_row = (mask & QT2_LAYOUT_ROW) != 0, do_col = (mask & QT2_LAYOUT_COL) != 0;
     RotViews out{};
@@ -536,7 +611,12 @@ qt2_status msed_enqueue_on_scratch(const void *x_bf16, int64_t rows, int64_t col
 
 extern "C" {
 
-int qt2_version(void) { return 100; }
+int qt2_version(void) { return 101; }
+
+void qt2_set_fault_hook(qt2_fault_hook hook, void *user) {
+    g_fault_user.store(user, std::memory_order_release);
+    g_fault_hook.store(hook, std::memory_order_release);
+}
 
 const char *qt2_status_string(qt2_status s) {
     switch (s) {
@@ -548,11 +628,13 @@ const char *qt2_status_string(qt2_status s) {
         case QT2_ERR_CUDA: return "CUDA error";
         case QT2_ERR_TIMEOUT: return "device-side wait timed out";
         case QT2_ERR_DEVICE: return "no sm_100 device";
+        case QT2_ERR_NONFINITE: return "input holds inf or NaN";
     }
     return "unknown status";
 }
 
 qt2_status qt2_device_status(qt2_stream_t stream, int *code) {
+    QT2_TRACE();
     if (!code) return QT2_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QT2_ERR_CUDA;
     int v = 0;
@@ -573,6 +655,7 @@ qt2_status qt2_quant_fwd46_workspace_size(int64_t rows, int64_t cols, size_t *by
 qt2_status qt2_quant_fwd46(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask,
                            const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
                            size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     (void)col_out;
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
@@ -600,6 +683,7 @@ qt2_status qt2_quant_msedEN(const void *x_bf16, int64_t rows, int64_t cols, int6
                             uint64_t seed, uint32_t tensor_id_row, uint32_t tensor_id_col,
                             const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
                             size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
     if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
@@ -629,6 +713,7 @@ qt2_status qt2_quant_sr_workspace_size(int64_t rows, int64_t cols, int layout_ma
 qt2_status qt2_quant_sr(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld, int layout_mask, uint64_t seed,
                         uint32_t tensor_id_row, uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
                         const qt2_nvfp4_view *col_out, void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
     if (layout_mask < 1 || layout_mask > 3) return QT2_ERR_INVALID_ARG;
@@ -648,6 +733,7 @@ qt2_status qt2_quant_sr(const void *x_bf16, int64_t rows, int64_t cols, int64_t 
 
 qt2_status qt2_gemm_nvfp4(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,
                           float alpha, void *c, int c_dtype, int64_t ldc, qt2_stream_t stream) {
+    QT2_TRACE();
     if (!a || !b || !c) return QT2_ERR_INVALID_ARG;
     if (c_dtype != QT2_DTYPE_BF16 && c_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
     if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K) || ldc < N) return QT2_ERR_SHAPE;
@@ -673,6 +759,7 @@ qt2_status qt2_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t
 
 qt2_status qt2_linear_fwd(const void *x, const void *w, int64_t M, int64_t K, int64_t N, void *y_bf16,
                           void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     if (!x || !w || !y_bf16) return QT2_ERR_INVALID_ARG;
     if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(w) || !aligned16(y_bf16)) return QT2_ERR_ALIGN;
@@ -700,6 +787,7 @@ qt2_status qt2_linear_bwd_workspace_size(int64_t M, int64_t K, int64_t N, size_t
 qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t M, int64_t K, int64_t N,
                           uint64_t seed, void *dx_bf16, void *dw, int dw_dtype, void *workspace, size_t ws_bytes,
                           qt2_stream_t stream) {
+    QT2_TRACE();
     if (!dy || !x || !w || !dx_bf16 || !dw) return QT2_ERR_INVALID_ARG;
     if (dw_dtype != QT2_DTYPE_BF16 && dw_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
     if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;
@@ -730,14 +818,19 @@ qt2_status qt2_linear_bwd(const void *dy, const void *x, const void *w, int64_t 
 }
 
 qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = check_device();
     if (st != QT2_OK) return st;
+    const int fa = fault_at("launch");
+    if (fa == kFaultFail) return QT2_ERR_CUDA;
+    if (fa == kFaultSkip) return QT2_OK;
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
     return from_cuda(cudaGetLastError());
 }
 
 qt2_status qt2_quant_fwd46_local(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                                  const qt2_nvfp4_view *row_out, qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
     if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
@@ -748,6 +841,7 @@ qt2_status qt2_quant_fwd46_local(const void *x_bf16, int64_t rows, int64_t cols,
 
 qt2_status qt2_gemm_nvfp4_local(const qt2_nvfp4_view *a, const qt2_nvfp4_view *b, int64_t M, int64_t N, int64_t K,
                                 float alpha, void *c, int c_dtype, int64_t ldc, qt2_stream_t stream) {
+    QT2_TRACE();
     if (!a || !b || !c) return QT2_ERR_INVALID_ARG;
     if (c_dtype != QT2_DTYPE_BF16 && c_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
     if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K) || ldc < N) return QT2_ERR_SHAPE;
@@ -772,6 +866,7 @@ qt2_status qt2_quant_fwd46_sq_workspace_size(int64_t rows, int64_t cols, size_t 
 qt2_status qt2_quant_fwd46_sq(const void *x_bf16, int64_t rows, int64_t cols, int64_t ld,
                               const qt2_nvfp4_view *row_out, const qt2_nvfp4_view *col_out, void *workspace,
                               size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
     if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
@@ -796,6 +891,7 @@ qt2_status qt2_quant_fwd46_msedEN_col(const void *x_bf16, int64_t rows, int64_t 
                                       uint32_t tensor_id_col, const qt2_nvfp4_view *row_out,
                                       const qt2_nvfp4_view *col_out, void *workspace, size_t ws_bytes,
                                       qt2_stream_t stream) {
+    QT2_TRACE();
     qt2_status st = validate_bf16(x_bf16, rows, cols, ld);
     if (st != QT2_OK) return st;
     if (!view_ok(row_out)) return row_out ? QT2_ERR_ALIGN : QT2_ERR_INVALID_ARG;
@@ -821,6 +917,7 @@ qt2_status qt2_linear_bwd_views_workspace_size(int64_t M, int64_t K, int64_t N, 
 qt2_status qt2_linear_bwd_views(const void *dy, int64_t M, int64_t K, int64_t N, uint64_t seed,
                                 const qt2_nvfp4_view *x_col, const qt2_nvfp4_view *w_col, void *dx_bf16, void *dw,
                                 int dw_dtype, void *workspace, size_t ws_bytes, qt2_stream_t stream) {
+    QT2_TRACE();
     if (!dy || !x_col || !w_col || !dx_bf16 || !dw) return QT2_ERR_INVALID_ARG;
     if (dw_dtype != QT2_DTYPE_BF16 && dw_dtype != QT2_DTYPE_F32) return QT2_ERR_INVALID_ARG;
     if (!dim_ok(M) || !dim_ok(K) || !dim_ok(N)) return QT2_ERR_SHAPE;

@@ -202,6 +202,13 @@ __device__ __forceinline__ uint32_t fwd46_group(const uint32_t (&w)[8], float g6
     return pick4 ? s4.code : s6.code;
 }
 
+// A max word (fp32 bits of max |x|, merged by integer max) that is inf or NaN: the input held
+// a non-finite value.  Recorded as QT2_ERR_NONFINITE; the outputs are then unspecified.
+__device__ __forceinline__ bool nonfinite_bits(uint32_t bits) { return bits >= 0x7F800000u; }
+__device__ __forceinline__ void check_finite_word(uint32_t bits) {
+    if (nonfinite_bits(bits)) set_device_error(QT2_ERR_NONFINITE);
+}
+
 // g = A/1792 of a tensor whose max |x| is A (1 for a zero tensor).
 __device__ __forceinline__ float fwd46_tensor_scale(const uint32_t *amax_word) {
     const float A = __uint_as_float(*amax_word);
@@ -269,8 +276,14 @@ __global__ void __launch_bounds__(256) fwd46_coop_kernel(const uint16_t *__restr
         __syncthreads();
         if (gave_up) return;
     }
-    // phase 2: the groups, one per thread and round, with the tensor's max
-    const float A = __uint_as_float(ld_acquire_gpu(&words[0]));
+    // phase 2: the groups, one per thread and round, with the tensor's max (inf or NaN in the
+    // input: reported, nothing quantized)
+    const uint32_t abits = ld_acquire_gpu(&words[0]);
+    if (nonfinite_bits(abits)) {
+        if (threadIdx.x == 0) set_device_error(QT2_ERR_NONFINITE);
+        return;
+    }
+    const float A = __uint_as_float(abits);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
     const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
@@ -349,6 +362,10 @@ __global__ void __cluster_dims__(kLocalCluster, 1, 1) __launch_bounds__(kLocalTh
 #pragma unroll
     for (int c = 0; c < kLocalCluster; ++c) bmax = max(bmax, ld_shared_cluster_u32(mapa_shared(smem_u32(&cta_max), c)));
     cluster_sync_all();   // no CTA leaves while a peer may still read its partial max
+    if (nonfinite_bits(bmax)) {   // inf or NaN in the block: reported, nothing quantized
+        if (threadIdx.x == 0) set_device_error(QT2_ERR_NONFINITE);
+        return;
+    }
     const float A = __uint_as_float(bmax);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
     const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
@@ -397,6 +414,10 @@ __global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restric
                                                        uint8_t *__restrict__ row_codes, uint8_t *__restrict__ row_scales,
                                                        float *__restrict__ row_g, uint8_t *__restrict__ col_codes,
                                                        uint8_t *__restrict__ col_scales, float *__restrict__ col_g) {
+    if (nonfinite_bits(*amax_word)) {   // inf or NaN in the input: reported, nothing quantized
+        if (blockIdx.x == 0 && threadIdx.x == 0) set_device_error(QT2_ERR_NONFINITE);
+        return;
+    }
     const float g = fwd46_tensor_scale(amax_word);
     const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -493,7 +514,9 @@ __global__ void __launch_bounds__(256) msed_finalize_kernel(FinalizeJob j0, Fina
     const bool second = (int64_t)blockIdx.x >= j0.blocks;
     const FinalizeJob &jb = second ? j1 : j0;
     const int64_t bid = second ? blockIdx.x - j0.blocks : blockIdx.x, nb = jb.blocks;
-    const float A = __uint_as_float(*jb.amax_word);
+    const uint32_t abits = *jb.amax_word;
+    if (bid == 0 && threadIdx.x == 0) check_finite_word(abits);   // max |y| is inf/NaN iff x was
+    const float A = __uint_as_float(abits);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kMsedDenominator) : 1.0f;
     const float ginv = __frcp_rn(g);
     if (bid == 0 && threadIdx.x == 0) *jb.tensor_scale = g;

@@ -21,7 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "qt2.h")
 
 QT2_OK = 0
 QT2_ERR_INVALID_ARG, QT2_ERR_SHAPE, QT2_ERR_ALIGN, QT2_ERR_WORKSPACE = -1, -2, -3, -4
-QT2_ERR_CUDA, QT2_ERR_TIMEOUT, QT2_ERR_DEVICE = -5, -6, -7
+QT2_ERR_CUDA, QT2_ERR_TIMEOUT, QT2_ERR_DEVICE, QT2_ERR_NONFINITE = -5, -6, -7, -8
 QT2_LAYOUT_ROW, QT2_LAYOUT_COL, QT2_LAYOUT_BOTH = 1, 2, 3
 QT2_DTYPE_BF16, QT2_DTYPE_F32 = 0, 1
 QT2_TID_SIGNS, QT2_TID_DY_ROW, QT2_TID_DY_COL, QT2_TID_W_COL, QT2_TID_X_COL = 0, 1, 2, 3, 4
@@ -31,6 +31,11 @@ class QT2Error(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
         super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+
+
+# qt2_set_fault_hook: int hook(const char *site, void *user); 0 = proceed, 1 = fail, 2 = skip
+FAULT_NONE, FAULT_FAIL, FAULT_SKIP = 0, 1, 2
+FaultHookC = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_char_p, ctypes.c_void_p)
 
 
 class NVFP4ViewC(ctypes.Structure):
@@ -72,6 +77,7 @@ def lib() -> ctypes.CDLL:
                 "qt2_linear_bwd": (i32, [vp, vp, vp, i64, i64, i64, u64, vp, vp, i32, vp, sz, vp]),
                 "qt2_quant_fwd46_local": (i32, [vp, i64, i64, i64, pv, vp]),
                 "qt2_selftest_wait_timeout": (i32, [vp]),
+                "qt2_set_fault_hook": (None, [FaultHookC, vp]),
                 "qt2_gemm_nvfp4_local": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
@@ -321,6 +327,29 @@ def qt2_gemm_nvfp4_local(a: View, b: View, M: int, N: int, K: int, alpha: float,
     ac, bc = a.c(), b.c()
     _check("qt2_gemm_nvfp4_local", lib().qt2_gemm_nvfp4_local(ctypes.byref(ac), ctypes.byref(bc), M, N, K, alpha,
                                                               _ptr(c), c_dtype, ldc, _stream(stream)))
+
+
+class fault_hook:
+    """Context manager around qt2_set_fault_hook: `decide(site) -> 0/1/2` is asked before every
+    CUDA call the library makes while enqueuing (FAULT_NONE, FAULT_FAIL, FAULT_SKIP); the
+    sites seen are recorded in `.sites`.  The hook is removed on exit."""
+
+    def __init__(self, decide):
+        self.decide, self.sites = decide, []
+
+        def _hook(site, _user):
+            name = site.decode()
+            self.sites.append(name)
+            return int(self.decide(name))
+        self._c = FaultHookC(_hook)   # kept alive while installed
+
+    def __enter__(self):
+        lib().qt2_set_fault_hook(self._c, None)
+        return self
+
+    def __exit__(self, *exc):
+        lib().qt2_set_fault_hook(FaultHookC(), None)
+        return False
 
 
 def qt2_selftest_wait_timeout(stream=None) -> None:

@@ -26,6 +26,56 @@ SHAPES = {
     "mlp8b_down": (16384, 14336, 4096),
 }
 
+# Workloads made of several linear layers: (name, M, K, N, x kind, dY kind, name of the linear
+# whose input X this one shares or None).  A shared X is the same tensor (gate and up read the
+# block's normalised hidden state).
+#   mlp8b      the Llama-3-8B MLP at 16384 tokens: gate and up 4096 -> 14336 on one X ~ N(0,1),
+#              down 14336 -> 4096 on X = SiLU(a) * b; dY rows log-normal (many tiny groups).
+#   stack1p1b  the linears of one 1.1B-class block (d_model 2048, 16 heads, FFN 5632) at 32768
+#              tokens: QKV 2048 -> 6144, O 2048 -> 2048, gate and up 2048 -> 5632 (shared X),
+#              down 5632 -> 2048 (SiLU-gated X); other inputs as llm1p9b.
+STACKS = {
+    "mlp8b": [("gate", 16384, 4096, 14336, "gauss", "lognormal_rows", None),
+              ("up", 16384, 4096, 14336, "gauss", "lognormal_rows", "gate"),
+              ("down", 16384, 14336, 4096, "silu_gated", "lognormal_rows", None)],
+    "stack1p1b": [("qkv", 32768, 2048, 6144, "t3_outlier_channels", "gauss_1e-4", None),
+                  ("o", 32768, 2048, 2048, "t3_outlier_channels", "gauss_1e-4", None),
+                  ("gate", 32768, 2048, 5632, "t3_outlier_channels", "gauss_1e-4", None),
+                  ("up", 32768, 2048, 5632, "t3_outlier_channels", "gauss_1e-4", "gate"),
+                  ("down", 32768, 5632, 2048, "silu_gated", "gauss_1e-4", None)],
+}
+_SINGLE_KINDS = {"tiny": ("gauss", "gauss1"), "llm1p9b": ("t3_outlier_channels", "gauss_1e-4"),
+                 "mlp8b_up": ("gauss", "lognormal_rows"), "mlp8b_down": ("silu_gated", "lognormal_rows")}
+
+
+def stack_linears(cfg: str):
+    """The linears of a workload as (name, M, K, N, x kind, dY kind, shared-X source)."""
+    if cfg in STACKS:
+        return list(STACKS[cfg])
+    M, K, N = SHAPES[cfg]
+    xk, dk = _SINGLE_KINDS[cfg]
+    return [(cfg, M, K, N, xk, dk, None)]
+
+
+def stack_inputs(cfg: str, seed: int = 0, device="cpu", only: str | None = None):
+    """{name: (X, W, dY)} for every linear of a workload (a single-linear config gives exactly
+    linear_inputs(cfg, seed)); linear i draws from sub-seeds seed + 10 i + {0, 1, 2}.  With
+    `only`, just that linear (and the one whose X it shares) is drawn."""
+    if cfg not in STACKS:
+        return {cfg: linear_inputs(cfg, seed, device)}
+    need = None
+    if only is not None:
+        src = {n: sh for n, *_, sh in STACKS[cfg]}
+        need = {only, src[only]}
+    out = {}
+    for i, (name, M, K, N, xk, dk, shared) in enumerate(STACKS[cfg]):
+        if need is not None and name not in need:
+            continue
+        s = seed + 10 * i
+        x = out[shared][0] if shared else make_x(M, K, xk, s, device)
+        out[name] = (x, make_w(N, K, s + 1, device=device), make_dy(M, N, dk, s + 2, device))
+    return out
+
 
 def _gen(device, seed: int) -> torch.Generator:
     g = torch.Generator(device=device)

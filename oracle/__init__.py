@@ -108,13 +108,20 @@ def _rows(fn, R: int, min_rows: int = 64):
 
 
 def _bf16_bits(x) -> np.ndarray:
-    """bf16 data as a C-contiguous uint16 array (accepts a uint16 array or a torch bf16 tensor)."""
+    """bf16 data as a C-contiguous uint16 array (accepts a uint16 array or a torch bf16 tensor).
+
+    The method is defined on real numbers only: a tensor holding inf or NaN (exponent field all
+    ones) is refused with ValueError, the counterpart of the library's QT2_ERR_NONFINITE."""
     if isinstance(x, np.ndarray):
         assert x.dtype == np.uint16
-        return np.ascontiguousarray(x)
-    import torch
-    assert x.dtype == torch.bfloat16
-    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+        b = np.ascontiguousarray(x)
+    else:
+        import torch
+        assert x.dtype == torch.bfloat16
+        b = np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    if np.any((b & 0x7F80) == 0x7F80):
+        raise ValueError("input holds inf or NaN: the quantizers are defined on finite values only")
+    return b
 
 
 # --------------------------------------------------------------------------- scalar formats
@@ -315,6 +322,8 @@ def msedEN(x, seed: int, tid: int, view: str = "row") -> View:
     _rows(lambda r0, r1: lib().or_msedEN_rows_stage1(_p(b), R, C, _p(sgn), r0, r1, _p(codes), _p(amax_g),
                                                      _p(P), _p(S)), R)
     A = float(amax_g.max()) if amax_g.size else 0.0
+    if not np.isfinite(A):
+        raise ValueError("the rotated values overflow binary32 (|x| above about 2^121)")
     g = lib().or_msedEN_tensor_scale(A)
     scales = np.zeros((R, C // 16), np.uint8)
     _rows(lambda r0, r1: lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r0, r1, _p(scales)), R)
@@ -361,6 +370,8 @@ def sr(x, seed: int, tid: int, view: str = "row") -> View:
     R, C = b.shape
     sgn = rht_signs(seed)
     A = rotated_amax(b, sgn)
+    if not np.isfinite(A):
+        raise ValueError("the rotated values overflow binary32 (|x| above about 2^121)")
     codes = np.zeros((R, C // 2), np.uint8)
     scales = np.zeros((R, C // 16), np.uint8)
     _rows(lambda r0, r1: lib().or_sr_rows(_p(b), R, C, _p(sgn), A, seed, tid, r0, r1, _p(codes), _p(scales)), R)

@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 24
+    assert len(names) == 25
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -40,7 +40,7 @@ def test_built_for_sm100a_only():
 
 def test_version_and_status_strings(L):
     assert qt2.qt2_version() >= 100
-    for code in range(0, -8, -1):
+    for code in range(0, -9, -1):
         s = qt2.qt2_status_string(code)
         assert s and s != "unknown status"
 
@@ -142,3 +142,84 @@ def test_scale_layout_helpers_are_inverse():
     assert np.array_equal(scales_to_canonical(canonical_to_scales(canon), R, C), canon)
     # one 512-byte atom holds 128 rows x 4 groups; rows r, r+32, r+64, r+96 share a 16-byte line
     assert off[0, 0] == 0 and off[32, 0] == 4 and off[1, 0] == 16 and off[0, 1] == 1 and off[0, 4] == 512
+
+
+# --------------------------------------------------------------------------- host-side fault injection
+def _skip_then_fail(fail_site):
+    """Skip every CUDA call before `fail_site` (no GPU is touched) and fail at it."""
+    return lambda site: qt2.FAULT_FAIL if site == fail_site else qt2.FAULT_SKIP
+
+
+def test_injected_launch_failure_returns_cuda_error(L):
+    """A launch that fails is reported as QT2_ERR_CUDA and nothing after it is enqueued; with
+    every other CUDA call skipped, no GPU is needed or touched."""
+    v = _view()
+    R = ctypes.byref
+    with qt2.fault_hook(_skip_then_fail("launch")) as h:
+        st = L.qt2_quant_msedEN(0x1000, 256, 256, 256, qt2.QT2_LAYOUT_BOTH, 1, 1, 2, R(v), R(v), 0x40000, 1 << 20,
+                                None)
+    assert st == qt2.QT2_ERR_CUDA
+    assert h.sites == ["device", "tensor_map", "memset", "launch"]   # the producer's launch failed first
+    with qt2.fault_hook(_skip_then_fail("launch")) as h:
+        st = L.qt2_quant_fwd46(0x1000, 128, 128, 128, 1, R(v), None, 0x40000, 256, None)
+    assert st == qt2.QT2_ERR_CUDA and h.sites == ["device", "memset", "launch"]
+    with qt2.fault_hook(_skip_then_fail("launch")) as h:
+        st = L.qt2_linear_bwd(0x1000, 0x2000, 0x3000, 256, 256, 256, 0, 0x4000, 0x5000, 1, 0x100000, 1 << 30, None)
+    assert st == qt2.QT2_ERR_CUDA and h.sites[-1] == "launch" and h.sites.count("launch") == 1
+    with qt2.fault_hook(_skip_then_fail("launch")):
+        assert L.qt2_selftest_wait_timeout(None) == qt2.QT2_ERR_CUDA
+
+
+def test_injected_failures_at_every_site_of_a_layer_call(L):
+    """Walk the layer's backward call through every CUDA call it makes: skipping all of them
+    completes with QT2_OK having touched nothing; failing the k-th one returns the error of that
+    site and stops there."""
+    R = ctypes.byref
+    args = (0x1000, 0x2000, 0x3000, 256, 256, 256, 0, 0x4000, 0x5000, 1, 0x100000, 1 << 30, None)
+    with qt2.fault_hook(lambda site: qt2.FAULT_SKIP) as h:
+        assert L.qt2_linear_bwd(*args) == qt2.QT2_OK
+    sites = list(h.sites)
+    # three MS-EDEN calls (descriptor, max reset, producer, scale pass) and two GEMMs (descriptors, launch)
+    assert sites.count("launch") == 8 and sites[0] == "device"
+    for k in range(len(sites)):
+        calls = []
+
+        def decide(site, k=k, calls=calls):
+            calls.append(site)
+            return qt2.FAULT_FAIL if len(calls) == k + 1 else qt2.FAULT_SKIP
+        with qt2.fault_hook(decide):
+            st = L.qt2_linear_bwd(*args)
+        assert len(calls) == k + 1, (k, calls)
+        assert st == (qt2.QT2_ERR_DEVICE if sites[k] == "device" else qt2.QT2_ERR_CUDA), (k, sites[k], st)
+    # the hook is gone: the plain call fails on the device query again (no GPU here) or runs
+    if not torch.cuda.is_available():
+        assert L.qt2_linear_bwd(*args) == qt2.QT2_ERR_DEVICE
+
+
+def test_injected_failure_of_the_noalloc_scratch_lookup(L):
+    v = _view()
+    R = ctypes.byref
+    with qt2.fault_hook(_skip_then_fail("symbol")) as h:
+        st = L.qt2_quant_msedEN_noalloc(0x1000, 256, 256, 256, qt2.QT2_LAYOUT_BOTH, 1, 1, 2, R(v), R(v), None)
+    assert st == qt2.QT2_ERR_CUDA and h.sites == ["device", "symbol"]
+
+
+# --------------------------------------------------------------------------- no-alloc capacity
+def test_noalloc_capacity_boundary(L):
+    """qt2_quant_msedEN_noalloc takes up to 32 MiB of pre-scales (rows*cols/4 bytes per view):
+    8192 x 8192 with both views and 8192 x 16384 with one view are accepted, one 128-block
+    more is refused with QT2_ERR_WORKSPACE before any CUDA call (fake addresses)."""
+    v = _view()
+    R = ctypes.byref
+    f = L.qt2_quant_msedEN_noalloc
+    # skip every CUDA call: an accepted call then enqueues nothing and returns QT2_OK
+    with qt2.fault_hook(lambda site: qt2.FAULT_SKIP):
+        assert f(0x1000, 8192, 8192, 8192, qt2.QT2_LAYOUT_BOTH, 1, 1, 2, R(v), R(v), None) == qt2.QT2_OK
+        assert f(0x1000, 8192, 16384, 16384, qt2.QT2_LAYOUT_ROW, 1, 1, 2, R(v), None, None) == qt2.QT2_OK
+        assert f(0x1000, 16384, 8192, 8192, qt2.QT2_LAYOUT_COL, 1, 1, 2, None, R(v), None) == qt2.QT2_OK
+        assert f(0x1000, 8192, 8320, 8320, qt2.QT2_LAYOUT_BOTH, 1, 1, 2, R(v), R(v), None) == qt2.QT2_ERR_WORKSPACE
+        assert f(0x1000, 8320, 8192, 8192, qt2.QT2_LAYOUT_BOTH, 1, 1, 2, R(v), R(v), None) == qt2.QT2_ERR_WORKSPACE
+        assert f(0x1000, 8192, 16512, 16512, qt2.QT2_LAYOUT_ROW, 1, 1, 2, R(v), None, None) == qt2.QT2_ERR_WORKSPACE
+    limit = 32 * 1024 * 1024
+    assert qt2.qt2_quant_msedEN_workspace_size(8192, 8192, qt2.QT2_LAYOUT_BOTH) == 256 + limit
+    assert qt2.qt2_quant_msedEN_workspace_size(8192, 16384, qt2.QT2_LAYOUT_ROW) == 256 + limit

@@ -87,3 +87,14 @@ def test_linear_bwd_views_matches_oracle(shape, seed):
         assert _rel(dw_g, dw_ref) < 1e-5
         _bound_check(dw_g, dw_ref,
                      O.gemm(np.abs(views["dy_col"].dequant()), np.abs(views["x_col"].dequant()), 2 ** -7), False)
+
+
+def test_fused_views_full_size():
+    """16384 x 8192 layer input with outlier channels (8192 tiles, ~55 per persistent CTA): the
+    forward view and the MS-EDEN column view from one read, bit-exact with the oracle."""
+    x = synth.make_x(16384, 8192, "t3_outlier_channels", 9)
+    seed, tid = 4242, qt2.QT2_TID_X_COL
+    vr, vc = gpu_fused(x, seed, tid)
+    _assert_view_equal(_host(vr, 16384, 8192), O.fwd46(x), "full-size forward view")
+    del vr
+    _assert_view_equal(_host(vc, 8192, 16384), O.msedEN(x, seed, tid, "col"), "full-size column view")

@@ -2,9 +2,10 @@
 against the oracle's fp64 results on the same seeded inputs.
 
 Small cases compare every output; the full-size cases (the 1.9B-class layer: tokens 16384,
-d_in 2048, d_out 8192, the launch configuration the benchmark times; the Llama-3-8B MLP gate/up
-4096 -> 14336 and down 14336 -> 4096 linears at 16384 tokens) compare sampled rows that the
-oracle computes one by one, plus bit-exact codes and scales of those rows."""
+d_in 2048, d_out 8192; the Llama-3-8B MLP gate/up 4096 -> 14336 and down 14336 -> 4096 linears
+at 16384 tokens, the launch configurations the benchmark times) compare every quantized view
+bit for bit with the oracle, and the GEMM outputs on sampled rows the oracle computes one by
+one from those views."""
 import numpy as np
 import pytest
 import torch
@@ -13,6 +14,7 @@ import oracle as O
 from nvfp4_quantized_b200 import qt2
 from nvfp4_quantized_b200 import synth
 from tests.layout import scales_to_canonical
+from tests.test_gpu_quant import _assert_view_equal
 
 pytestmark = pytest.mark.gpu
 
@@ -75,54 +77,77 @@ def test_linear_bwd_bf16_dw():
     assert _rel(dw.float().cpu().numpy().astype(np.float64), dw_ref) < 4e-3
 
 
-def _view_rows(view: qt2.View, rows, R, C):
-    codes = view.codes[torch.from_numpy(rows).cuda()].cpu().numpy()
-    scales = scales_to_canonical(view.scales.cpu().numpy(), R, C)[rows]
-    return codes, scales, np.float32(view.tensor_scale.item())
+def _full_view(view: qt2.View, R, C):
+    return (view.codes.cpu().numpy(), scales_to_canonical(view.scales.cpu().numpy(), R, C),
+            np.float32(view.tensor_scale.item()))
 
 
 @pytest.mark.parametrize("config", ["llm1p9b", "mlp8b_up", "mlp8b_down"])
-def test_full_size_sampled(config):
-    """Full-size layer: sampled rows of Y, dX and dW against the oracle, and bit-exact
-    codes/scales of the sampled rows of every quantized view."""
+def test_full_size_views_and_layer(config):
+    """Full-size layer in the launch configuration the benchmark times: EVERY code, scale and
+    tensor scale of every quantized view (forward views of X and W, MS-EDEN views of dY both
+    ways, W's and X's column views) equals the oracle's; Y, dX and dW of the layer call match
+    the oracle's fp64 products of those views on sampled rows.  At these sizes every
+    persistent producer wraps its tile ring many times per CTA and the forward quantizer's
+    grid-stride loop covers millions of groups per launch."""
     M, K, N = synth.SHAPES[config]
     x, w, dy = synth.linear_inputs(config, 0)
     seed = 2024
     y, dx, dw = run_linear(x, w, dy, seed)
+    xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
     rng = np.random.default_rng(0)
     rows_m = np.sort(rng.choice(M, 6, replace=False))
     rows_n = np.sort(rng.choice(N, 6, replace=False))
 
-    # forward: X rows via the oracle's row-range quantizer with the full-tensor max; W in full
-    vx_full = O.fwd46(x)       # all rows (cheap enough: 33M elements)
-    vw = O.fwd46(w)
-    y_ref = O.gemm(vx_full.dequant_rows(rows_m), vw.dequant(), 1.0)
+    # forward views, full tensors (the calls qt2_linear_fwd makes)
+    def fwd_view(t, R, C):
+        v = qt2.alloc_view(R, C)
+        ws = qt2.alloc_workspace(qt2.qt2_quant_fwd46_workspace_size(R, C))
+        qt2.qt2_quant_fwd46(t, R, C, C, qt2.QT2_LAYOUT_ROW, v, None, ws, ws.numel())
+        assert qt2.qt2_device_status() == 0
+        return _full_view(v, R, C)
+
+    o_x = O.fwd46(x)
+    _assert_view_equal(fwd_view(xd, M, K), o_x, f"{config} fwd46 X")
+    o_w = O.fwd46(w)
+    _assert_view_equal(fwd_view(wd, N, K), o_w, f"{config} fwd46 W")
+    y_ref = O.gemm(o_x.dequant_rows(rows_m), o_w.dequant(), 1.0)
     y_g = y[torch.from_numpy(rows_m).cuda()].float().cpu().numpy().astype(np.float64)
     assert _rel(y_g, y_ref) < 4e-3
+    _bound_check(y_g, y_ref, O.gemm(np.abs(o_x.dequant_rows(rows_m)), np.abs(o_w.dequant()), 1.0), True)
+    del o_x, o_w
 
-    # standalone quantizers at full size, same launch configuration as inside the layer
-    xd, wd, dyd = x.cuda(), w.cuda(), dy.cuda()
-    v_dy_row, v_dy_col = qt2.alloc_view(M, N), qt2.alloc_view(N, M)
-    ws = qt2.alloc_workspace(qt2.qt2_quant_msedEN_workspace_size(M, N, qt2.QT2_LAYOUT_BOTH))
-    qt2.qt2_quant_msedEN(dyd, M, N, N, qt2.QT2_LAYOUT_BOTH, seed, qt2.QT2_TID_DY_ROW, qt2.QT2_TID_DY_COL, v_dy_row,
-                         v_dy_col, ws, ws.numel())
-    assert qt2.qt2_device_status() == 0
+    # MS-EDEN views, full tensors (the calls qt2_linear_bwd makes)
+    def msed_views(t, R, C, mask, tid_row, tid_col):
+        vr = qt2.alloc_view(R, C) if mask & 1 else None
+        vc = qt2.alloc_view(C, R) if mask & 2 else None
+        ws = qt2.alloc_workspace(qt2.qt2_quant_msedEN_workspace_size(R, C, mask))
+        qt2.qt2_quant_msedEN(t, R, C, C, mask, seed, tid_row, tid_col, vr, vc, ws, ws.numel())
+        assert qt2.qt2_device_status() == 0
+        return (_full_view(vr, R, C) if vr is not None else None, _full_view(vc, C, R) if vc is not None else None)
 
+    g_dy_row, g_dy_col = msed_views(dyd, M, N, qt2.QT2_LAYOUT_BOTH, qt2.QT2_TID_DY_ROW, qt2.QT2_TID_DY_COL)
     o_dy_row = O.msedEN(dy, seed, qt2.QT2_TID_DY_ROW, "row")
+    _assert_view_equal(g_dy_row, o_dy_row, f"{config} MS-EDEN dY row")
+    del g_dy_row
+    _, g_w_col = msed_views(wd, N, K, qt2.QT2_LAYOUT_COL, 0, qt2.QT2_TID_W_COL)
     o_w_col = O.msedEN(w, seed, qt2.QT2_TID_W_COL, "col")
-    got = _view_rows(v_dy_row, rows_m, M, N)
-    assert got[2] == o_dy_row.g
-    assert np.array_equal(got[0], o_dy_row.codes[rows_m]) and np.array_equal(got[1], o_dy_row.scales[rows_m])
+    _assert_view_equal(g_w_col, o_w_col, f"{config} MS-EDEN W col")
+    del g_w_col
     dx_ref = O.gemm(o_dy_row.dequant_rows(rows_m), o_w_col.dequant(), 2.0 ** -7)
     dx_g = dx[torch.from_numpy(rows_m).cuda()].float().cpu().numpy().astype(np.float64)
     assert _rel(dx_g, dx_ref) < 4e-3
-    del o_dy_row
+    _bound_check(dx_g, dx_ref, O.gemm(np.abs(o_dy_row.dequant_rows(rows_m)), np.abs(o_w_col.dequant()), 2.0 ** -7),
+                 True)
+    del o_dy_row, o_w_col
 
     o_dy_col = O.msedEN(dy, seed, qt2.QT2_TID_DY_COL, "col")
+    _assert_view_equal(g_dy_col, o_dy_col, f"{config} MS-EDEN dY col")
+    del g_dy_col
+    _, g_x_col = msed_views(xd, M, K, qt2.QT2_LAYOUT_COL, 0, qt2.QT2_TID_X_COL)
     o_x_col = O.msedEN(x, seed, qt2.QT2_TID_X_COL, "col")
-    got = _view_rows(v_dy_col, rows_n, N, M)
-    assert got[2] == o_dy_col.g
-    assert np.array_equal(got[0], o_dy_col.codes[rows_n]) and np.array_equal(got[1], o_dy_col.scales[rows_n])
+    _assert_view_equal(g_x_col, o_x_col, f"{config} MS-EDEN X col")
+    del g_x_col
     dw_ref = O.gemm(o_dy_col.dequant_rows(rows_n), o_x_col.dequant(), 2.0 ** -7)
     dw_g = dw[torch.from_numpy(rows_n).cuda()].cpu().numpy().astype(np.float64)
     assert _rel(dw_g, dw_ref) < 1e-5

@@ -65,3 +65,15 @@ def test_msedEN_beats_sr_on_gpu_outputs():
 def _rotated_target(x, seed):
     from tests.test_oracle_msedEN import _rotated
     return _rotated(x, seed).astype(np.float64)
+
+
+def test_sr_full_size_both_views():
+    """16384 x 8192 (8192 tiles: every persistent CTA wraps the tile ring ~55 times), both
+    views, log-normal rows (many groups far below the tensor max): bit-exact with the oracle."""
+    from nvfp4_quantized_b200 import synth
+    x = synth.make_dy(16384, 8192, "lognormal_rows", 5)
+    seed = 0xC0FFEE
+    got = gpu_sr(x, seed, 21, 22, qt2.QT2_LAYOUT_BOTH)
+    _assert_view_equal(got["row"], O.sr(x, seed, 21, "row"), "full-size SR row")
+    del got["row"]
+    _assert_view_equal(got["col"], O.sr(x, seed, 22, "col"), "full-size SR col")

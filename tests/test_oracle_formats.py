@@ -177,3 +177,34 @@ def test_rht_signs_follow_word_bits():
             bit = (words[i >> 5] >> (i & 31)) & 1
             assert s[i] == (-1.0 if bit else 1.0)
         assert 30 < int((s < 0).sum()) < 98
+
+
+def test_nonfinite_inputs_are_refused():
+    """The quantizers are defined on finite values: inf or NaN anywhere in the input is refused
+    (the library reports the same inputs as QT2_ERR_NONFINITE)."""
+    import pytest
+    import torch
+    for bad in (float("inf"), float("-inf"), float("nan")):
+        x = torch.zeros((128, 128), dtype=torch.bfloat16)
+        x[5, 77] = bad
+        for fn in (lambda t: O.fwd46(t), lambda t: O.msedEN(t, 1, 1, "row"), lambda t: O.msedEN(t, 1, 2, "col"),
+                   lambda t: O.sr(t, 1, 1, "row"), lambda t: O.fwd46_sq(t), lambda t: O.fwd46_local(t)):
+            with pytest.raises(ValueError):
+                fn(x)
+    # the largest finite bf16 is accepted
+    x = torch.full((128, 128), 3.3895313892515355e38, dtype=torch.bfloat16)
+    assert np.isfinite(O.fwd46(x).g)
+
+
+def test_rotation_overflow_is_refused():
+    """Finite inputs whose 128-point rotation overflows binary32 are refused by the rotating
+    quantizers (the library reports them as QT2_ERR_NONFINITE); the forward quantizer, which
+    does not rotate, takes them."""
+    import pytest
+    import torch
+    x = torch.full((128, 128), 2.0 ** 125, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        O.msedEN(x, 1, 1, "row")
+    with pytest.raises(ValueError):
+        O.sr(x, 1, 1, "row")
+    assert np.isfinite(O.fwd46(x).g)

@@ -74,6 +74,23 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     _same(a_c, b_c)
 
 
+@pytest.mark.gpu
+def test_noalloc_at_the_largest_accepted_size():
+    """8192 x 8192 with both views fills the built-in scratch exactly: the results are the
+    workspace entry point's, bit for bit, on two calls in a row (the second with a smaller input,
+    so a view maximum left over from the first would change its scales)."""
+    g = torch.Generator(device="cuda").manual_seed(7)
+    for seed, scale in ((21, 1.0), (22, 1e-3)):
+        x = (torch.randn((8192, 8192), generator=g, device="cuda") * scale).to(torch.bfloat16)
+        got_r, got_c = _noalloc(x, 8192, 8192, qt2.QT2_LAYOUT_BOTH, seed, 1, 2)
+        ref_r, ref_c = _with_workspace(x, 8192, 8192, qt2.QT2_LAYOUT_BOTH, seed, 1, 2)
+        torch.cuda.synchronize()
+        assert qt2.qt2_device_status() == 0
+        _same(got_r, ref_r)
+        _same(got_c, ref_c)
+        del x, got_r, got_c, ref_r, ref_c
+
+
 def test_noalloc_rejects_tensors_beyond_the_builtin_scratch():
     """A tensor whose scratch would not fit in the built-in array is refused before any work
     (fake, never-dereferenced device addresses: the check runs on the host first)."""
