@@ -68,6 +68,7 @@ def lib():
                 "or_fwd46_rows": (None, [vp, i64, i64, f32, i64, i64, vp, vp, vp, vp, vp]),
                 "or_fwd46_sq_blocks": (None, [vp, i64, i64, f32, i64, i64, vp, vp, vp, vp, vp]),
                 "or_msedEN_rows_stage1": (None, [vp, i64, i64, vp, i64, i64, vp, vp, vp, vp]),
+                "or_msedEN_rotated_stage1": (None, [vp, i64, i64, i64, i64, vp, vp, vp, vp]),
                 "or_msedEN_tensor_scale": (f32, [f32]),
                 "or_msedEN_finalize": (None, [vp, i64, i64, f32, u64, u32, i64, i64, vp]),
                 "or_dequant": (None, [vp, vp, i64, i64, f32, i64, i64, vp]),
@@ -328,6 +329,28 @@ def msedEN(x, seed: int, tid: int, view: str = "row") -> View:
     scales = np.zeros((R, C // 16), np.uint8)
     _rows(lambda r0, r1: lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r0, r1, _p(scales)), R)
     return View(codes, scales, g, amax=np.float32(A), P=P, S=S, amax_g=amax_g, signs=sgn)
+
+
+def msedEN_rotated(y: np.ndarray, seed: int, tid: int) -> View:
+    """The MS-EDEN steps on values that are already rotated (fp32 [R][C], C a multiple of 128),
+    e.g. by a uniformly random orthogonal map instead of the randomized Hadamard: group scales,
+    RTN codes, the EDEN factor per 128-block, the view's tensor scale and the stochastically
+    rounded E4M3 scales -- everything msedEN does after its rotation."""
+    yf = np.ascontiguousarray(y, dtype=np.float32)
+    R, C = yf.shape
+    codes = np.zeros((R, C // 2), np.uint8)
+    amax_g = np.zeros((R, C // 16), np.float32)
+    P = np.zeros((R, C // 16), np.float32)
+    S = np.zeros((R, C // 128), np.float32)
+    _rows(lambda r0, r1: lib().or_msedEN_rotated_stage1(_p(yf), R, C, r0, r1, _p(codes), _p(amax_g), _p(P), _p(S)),
+          R)
+    A = float(amax_g.max()) if amax_g.size else 0.0
+    if not np.isfinite(A):
+        raise ValueError("non-finite rotated values")
+    g = lib().or_msedEN_tensor_scale(A)
+    scales = np.zeros((R, C // 16), np.uint8)
+    _rows(lambda r0, r1: lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r0, r1, _p(scales)), R)
+    return View(codes, scales, g, amax=np.float32(A), P=P, S=S, amax_g=amax_g)
 
 
 def unrotate(y: np.ndarray, seed: int) -> np.ndarray:

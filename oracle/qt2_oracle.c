@@ -350,14 +350,53 @@ OR_EXPORT void or_fwd46_sq_blocks(const uint16_t *x, int64_t R, int64_t C, float
 }
 
 /* ------------------------------------------------------------------ backward: MS-EDEN */
-/* Stage 1 of MS-EDEN over rows [r0, r1) of a bf16 [R][C] matrix grouped along C (C a multiple
- * of 128).  Per 128-block ([QII-tg] "Method", item 1; [QII-ru] "Unbiased quantization with MS-EDEN"):
- *   y = H D x (randomized Hadamard rotation);
+/* The EDEN steps on one rotated 128-block y ([QII-tg] "Method", item 1; [QII-ru] "Unbiased
+ * quantization with MS-EDEN"):
  *   per 16-group: a = max|y|, p = a/6, codes = RTN_E2M1(y * (1/p)),
  *                 t = sum val(code)*y, n = sum y*y;
  *   per block:    S = sum n / sum p*t  (the EDEN factor <x,x>/<Q(Rx),Rx>, taken in the
- *                 rotated domain where both inner products are 128x the original ones);
+ *                 rotated domain, where both inner products are those of x up to the same
+ *                 constant factor of the rotation's normalisation);
  *   pre-scale P = S * p per group.
+ * Writes the block's 64 code bytes, 8 group maxima and 8 pre-scales; returns S. */
+static float or_eden_block(const float y[128], uint8_t codes[64], float amax_g[8], float P[8])
+{
+    float nq[8], ptq[8], pq[8];
+    uint8_t cq[128];
+    for (int q = 0; q < 8; q++) {
+        const float *yq = y + 16 * q;
+        float a = 0.0f;
+        for (int i = 0; i < 16; i++) if (fabsf(yq[i]) > a) a = fabsf(yq[i]);
+        amax_g[q] = a;
+        float tv[16], nv[16];
+        if (!(a >= OR_TINY)) {
+            pq[q] = 0.0f;
+            for (int i = 0; i < 16; i++) cq[16 * q + i] = signbit(yq[i]) ? 8 : 0;
+            nq[q] = 0.0f;
+            ptq[q] = 0.0f;
+            continue;
+        }
+        float p = a / 6.0f;
+        float rcp = 1.0f / p;
+        for (int i = 0; i < 16; i++) {
+            uint8_t c = or_e2m1_encode(yq[i] * rcp);
+            cq[16 * q + i] = c;
+            tv[i] = or_e2m1_value(c) * yq[i];
+            nv[i] = yq[i] * yq[i];
+        }
+        pq[q] = p;
+        nq[q] = or_tree(nv, 16);
+        ptq[q] = p * or_tree(tv, 16);
+    }
+    float num = or_tree(nq, 8), den = or_tree(ptq, 8);
+    float S = den > 0.0f ? num / den : 1.0f;
+    for (int q = 0; q < 8; q++) P[q] = S * pq[q];
+    for (int i = 0; i < 64; i++) codes[i] = (uint8_t)(cq[2 * i] | (cq[2 * i + 1] << 4));
+    return S;
+}
+
+/* Stage 1 of MS-EDEN over rows [r0, r1) of a bf16 [R][C] matrix grouped along C (C a multiple
+ * of 128): per 128-block the randomized Hadamard rotation y = H D x, then the EDEN steps above.
  * Outputs: codes [R][C/2], amax_g [R][C/16] (= a), P [R][C/16], S [R][C/128] (nullable). */
 OR_EXPORT void or_msedEN_rows_stage1(const uint16_t *x, int64_t R, int64_t C, const float sgn[128],
                                      int64_t r0, int64_t r1, uint8_t *codes, float *amax_g,
@@ -370,41 +409,27 @@ OR_EXPORT void or_msedEN_rows_stage1(const uint16_t *x, int64_t R, int64_t C, co
             float y[128];
             for (int i = 0; i < 128; i++) y[i] = sgn[i] * or_bf16_to_f32(x[r * C + b * 128 + i]);
             or_fwht128(y);
-            float nq[8], ptq[8], pq[8];
-            uint8_t cq[128];
-            for (int q = 0; q < 8; q++) {
-                const float *yq = y + 16 * q;
-                float a = 0.0f;
-                for (int i = 0; i < 16; i++) if (fabsf(yq[i]) > a) a = fabsf(yq[i]);
-                amax_g[r * G + b * 8 + q] = a;
-                float tv[16], nv[16];
-                if (!(a >= OR_TINY)) {
-                    pq[q] = 0.0f;
-                    for (int i = 0; i < 16; i++) cq[16 * q + i] = signbit(yq[i]) ? 8 : 0;
-                    nq[q] = 0.0f;
-                    ptq[q] = 0.0f;
-                    continue;
-                }
-                float p = a / 6.0f;
-                float rcp = 1.0f / p;
-                for (int i = 0; i < 16; i++) {
-                    uint8_t c = or_e2m1_encode(yq[i] * rcp);
-                    cq[16 * q + i] = c;
-                    tv[i] = or_e2m1_value(c) * yq[i];
-                    nv[i] = yq[i] * yq[i];
-                }
-                pq[q] = p;
-                nq[q] = or_tree(nv, 16);
-                ptq[q] = p * or_tree(tv, 16);
-            }
-            float num = or_tree(nq, 8), den = or_tree(ptq, 8);
-            float S = den > 0.0f ? num / den : 1.0f;
+            float S = or_eden_block(y, codes + r * (C / 2) + b * 64, amax_g + r * G + b * 8, P + r * G + b * 8);
             if (S_out) S_out[r * (C / 128) + b] = S;
-            for (int q = 0; q < 8; q++) P[r * G + b * 8 + q] = S * pq[q];
-            for (int i = 0; i < 64; i++)
-                codes[r * (C / 2) + b * 64 + i] = (uint8_t)(cq[2 * i] | (cq[2 * i + 1] << 4));
         }
     }
+}
+
+/* The same EDEN steps on values already rotated by some other orthogonal map (fp32 [R][C], C a
+ * multiple of 128): used to separate the EDEN steps' own unbiasedness from that of the
+ * 128-point randomized Hadamard rotation (EDEN is exactly unbiased for a uniformly random
+ * rotation).  Outputs as or_msedEN_rows_stage1. */
+OR_EXPORT void or_msedEN_rotated_stage1(const float *y, int64_t R, int64_t C, int64_t r0, int64_t r1,
+                                        uint8_t *codes, float *amax_g, float *P, float *S_out)
+{
+    (void)R;
+    int64_t G = C / 16;
+    for (int64_t r = r0; r < r1; r++)
+        for (int64_t b = 0; b < C / 128; b++) {
+            float S = or_eden_block(y + r * C + b * 128, codes + r * (C / 2) + b * 64, amax_g + r * G + b * 8,
+                                    P + r * G + b * 8);
+            if (S_out) S_out[r * (C / 128) + b] = S;
+        }
 }
 
 /* Tensor scale of an MS-EDEN view: g = A / (6*256) with A = max|y| over the view, leaving

@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 import oracle as O
-from tests.test_oracle_msedEN import _bf16, _mean_stats, _rotated, _unpack
+from tests.test_oracle_msedEN import _bf16, _bias_inputs, _mean_stats, _rotated, _unpack, strict_unbiased
 
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
@@ -46,11 +46,12 @@ def test_neighbours_and_no_clipping():
 
 
 def test_unbiased_over_2048_seeds():
-    rng = np.random.default_rng(9)
-    x = _bf16(rng.standard_normal((2, 256)))
-    xd = x.float().numpy().astype(np.float64)
+    """The binary32 SR quantizer is unbiased up to binary32 rounding of d, 1/d and |y|*r (relative
+    2^-23, far below what 2048 seeds resolve): the strict per-coordinate bar on 2048
+    coordinates, one of them an outlier."""
+    x, xd = _bias_inputs()
     z, rel_bias, rel_noise = _mean_stats(lambda s: O.unrotate(O.sr(x, s, 7, "row").dequant(), s), xd, 2048)
-    assert np.mean(np.abs(z) > 3) <= 0.03 and rel_bias < 0.05 * rel_noise
+    strict_unbiased(z, "SR baseline (binary32)")
 
 
 def test_agrees_with_fp64_baseline():
