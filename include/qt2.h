@@ -309,6 +309,20 @@ QT2_API qt2_status qt2_linear_bwd_views(const void *dy, int64_t M, int64_t K, in
  * --------------------------------------------------------------------------------------- */
 QT2_API qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Self-test of the quantizers' division shortcuts (the method's group scales need RN(a/6) and
+ * RN(1/p) in binary32; the kernels form them with fused multiply-adds): for every binary32
+ * value whose biased exponent lies in [exp_lo, exp_hi] (1 <= exp_lo <= exp_hi <= 254, every
+ * significand), compares the kernels' reciprocal with the IEEE reciprocal and their division by
+ * 6 with the IEEE quotient, and adds the numbers of mismatching results to mismatches[0]
+ * (reciprocal) and mismatches[1] (division by 6): two device counters, 8-byte aligned, zeroed
+ * by the caller.  The kernels use the reciprocal on group scales p in [2^-103, 2^126) (biased
+ * exponents 24..252) and the division on group maxima in [2^-100, 2^128) (27..254).
+ * Enqueued on `stream`.
+ * --------------------------------------------------------------------------------------- */
+QT2_API qt2_status qt2_selftest_division(uint32_t exp_lo, uint32_t exp_hi, unsigned long long *mismatches,
+                                         qt2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,13 +19,17 @@
 // Design: persistent CTAs of 512 threads (16 warps at up to 128 registers, so an SM keeps 16
 // warps in flight), 128x128 bf16 tiles streamed by TMA (128-byte swizzle) through a 3-deep ring.
 // Two threads (adjacent lanes, h = 0, 1) share one 128-element vector: thread h holds elements
-// [64h, 64h + 64) as 32 packed pairs and runs the butterfly strides 1..32 in registers; stride 64
-// crosses the pair with one shuffle per packed value.  After it, thread h owns the 16-groups
+// [64h, 64h + 64) in 32 packed fp32 pairs and runs the butterfly strides 1..32 in registers;
+// stride 64 crosses the pair with one shuffle per packed value.  A pair register holds elements
+// k and k + 8 (the two halves of one 16-group), so every butterfly stage but stride 8 and every
+// level but the last of the 16-term group trees run on packed f32x2 instructions.  Register
+// slot m holds element k = (m & 7) | ((m >> 3) & 1) << 4 | (((m >> 4) & 1) ^ h) << 5 of the
+// thread's half (and k + 8): thread 1 keeps its two 32-element quarters swapped, so that the
+// cross step is the same instructions on both threads -- it turns thread 1's stride-32 and
+// stride-64 subtractions around, and an FMA with sigma = +-1 gives each thread its own operand
+// order exactly (signed zeros included).  After the butterfly thread h owns the 16-groups
 // {2h, 2h+1} and {4+2h, 5+2h} of the block and quantizes them; the block sums for S meet
-// through two more shuffles.  To make the cross step the same instructions on both threads,
-// thread 1 keeps its half with the two 32-element quarters swapped (natural pair n of its half
-// sits in slot (n + 16) % 32); that turns its stride-32 and stride-64 subtractions around, and
-// an FMA with sigma = +-1 gives each thread its own operand order exactly (signed zeros included).
+// through two more shuffles.
 //   both views : warps 0..7 take the rows of each tile, warps 8..15 its columns;
 //   one view   : warps 0..7 and 8..15 take alternate tiles.
 // A ring stage is refilled by the last warp that has read it (a shared counter), so the two
@@ -110,16 +114,25 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     return v;
 }
 
-// Butterfly strides 2..64 and quantization of one vector held by a thread pair.
-// In: P = the thread's half after stride 1, in slot order; sg = (sigma, sigma), nsg = -sg with
-// sigma = +1 on thread 0 and -1 on thread 1.
-// Out: cw[2g], cw[2g+1] = codes of local group g (element 8w+i of the group in nibble i of
-// word w); Pq[g] = S * p of local group g.  Local groups 0, 1, 2, 3 are the block's groups 2h,
-// 2h+1, 4+2h, 5+2h.  amax = running max |y|.
+// RN(1/p) for normal p (2^-103 <= p < 2^126, so 1/p is normal): the hardware approximation y,
+// then one correction y + y*(1 - p*y) with both steps fused multiply-adds (Markstein's
+// reciprocal iteration, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34, 1990).  Checked bit for bit against the IEEE reciprocal over
+// every significand of several binades (qt2_selftest_rcp).
+__device__ __forceinline__ float rcp_rn(float p) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(p));
+    const float e = __fmaf_rn(-p, y, 1.0f);
+    return __fmaf_rn(y, e, y);
+}
+
+// Butterfly strides 2..64 of one vector held by a thread pair (stride 1 is taken as the tile is
+// read).  In: P = the thread's half in slot order (see the layout above); sg = (sigma, sigma),
+// nsg = -sg with sigma = +1 on thread 0 and -1 on thread 1.
 __device__ __forceinline__ void rotate_tail(uint64_t (&P)[32], uint64_t sg, uint64_t nsg) {
-    // strides 2, 4, 8, 16: slots j and j + hp of the same 16-slot half, same order on both threads
+    // strides 2, 4 (slot bits 1, 2): same order on both threads
 #pragma unroll
-    for (int hp = 1; hp < 16; hp <<= 1) {
+    for (int hp = 2; hp <= 4; hp <<= 1) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             if ((j & hp) == 0) {
@@ -129,7 +142,24 @@ __device__ __forceinline__ void rotate_tail(uint64_t (&P)[32], uint64_t sg, uint
             }
         }
     }
-    // stride 32: thread 0 forms (u + v, u - v), thread 1 (its halves swapped) (v - u, v + u)
+    // stride 8: the two halves of each pair register
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float lo, hi;
+        f2_split(P[j], lo, hi);
+        P[j] = f2(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+    }
+    // stride 16 (slot bit 3)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if ((j & 8) == 0) {
+            const uint64_t a = P[j], b = P[j + 8];
+            P[j] = f2_add(a, b);
+            P[j + 8] = f2_sub(a, b);
+        }
+    }
+    // stride 32 (slot bit 4): thread 0 forms (u + v, u - v), thread 1 (its quarters swapped)
+    // (v - u, v + u)
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
         const uint64_t u = P[j], v = P[j + 16];
@@ -137,7 +167,7 @@ __device__ __forceinline__ void rotate_tail(uint64_t (&P)[32], uint64_t sg, uint
         P[j + 16] = f2_fma(nsg, v, u);
     }
     // stride 64 across the pair: both threads send slot 16 + k and keep slot k.  Thread 0 keeps
-    // z[2k] and receives z[64 + 2k]; thread 1 keeps z[96 + 2k] and receives z[32 + 2k].
+    // the elements with bit 5 clear and receives thread 1's; thread 1 the other way round.
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
         const uint64_t recv = shfl_xor1_u64(P[16 + k]);
@@ -147,58 +177,59 @@ __device__ __forceinline__ void rotate_tail(uint64_t (&P)[32], uint64_t sg, uint
     }
 }
 
-__device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint64_t nsg, uint32_t (&cw)[8],
-                                            float (&Pq)[4], float &amax) {
+// The 16 values of local group g (0..3) after rotate_tail: element i of the group is the low
+// half of slot 8g + i for i < 8 and the high half of slot 8g + i - 8 for i >= 8.  Local groups
+// 0, 1, 2, 3 are the block's groups 2h, 2h+1, 4+2h, 5+2h.
+__device__ __forceinline__ void group_values(const uint64_t (&P)[32], int g, float (&y)[16]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f2_split(P[8 * g + i], y[i], y[i + 8]);
+}
+
+// max |y| of a group (NaN-propagating, see absmax3)
+__device__ __forceinline__ float group_absmax(const float (&y)[16]) {
+    const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
+    const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
+    const float m4 = absmax3(y[12], y[13], y[14]);
+    return max2n(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+}
+
+// Quantization of the thread's four local groups after rotate_tail.
+// Out: cw[2g], cw[2g+1] = codes of local group g (element 8w+i of the group in nibble i of
+// word w); Pq[g] = S * p of local group g.  amax = running max |y|.
+__device__ __forceinline__ void msed_vector(uint64_t (&P)[32], uint64_t sg, uint64_t nsg, uint64_t nz,
+                                            uint32_t (&cw)[8], float (&Pq)[4], float &amax) {
     rotate_tail(P, sg, nsg);
 
     float nq[4], ptq[4], pq[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         float y[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f2_split(P[8 * g + i], y[2 * i], y[2 * i + 1]);
-        // max is exact: the evaluation order does not matter
-        const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
-        const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
-        const float m4 = absmax3(y[12], y[13], y[14]);
-        const float a = max2n(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+        group_values(P, g, y);
+        const float a = group_absmax(y);
         amax = max2n(amax, a);
         const bool live = a >= kTiny;
         const float p = live ? div6_rn(a) : 0.0f;
-        const float r = live ? __frcp_rn(p) : 0.0f;          // flushed group: sign-preserving zeros
+        const float r = live ? rcp_rn(p) : 0.0f;          // flushed group: sign-preserving zeros
         const uint64_t rr = f2(r, r);
         float v[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f2_split(f2_mul(P[8 * g + i], rr), v[2 * i], v[2 * i + 1]);
-        float val[16];
+        for (int i = 0; i < 8; ++i) f2_split(f2_mul(P[8 * g + i], rr), v[i], v[i + 8]);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float vh[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) vh[i] = v[8 * hh + i];
             cw[2 * g + hh] = e2m1x8(vh);
-            float dv[8];
-            e2m1x8_values(cw[2 * g + hh], dv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) val[8 * hh + i] = dv[i];
         }
-        // products val*y and y*y, then the 16-term trees; level 1 pairs adjacent elements,
-        // levels 2..4 run on (t, n) packed together
-        uint64_t tn[8];
+        // products val*y and y*y on the pairs (i, i + 8), then the 16-term trees
+        uint64_t T[8], N[8];
+        e2m1x16_pairs(cw[2 * g], cw[2 * g + 1], T);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float t0, t1, n0, n1;
-            f2_split(f2_mul(f2(val[2 * i], val[2 * i + 1]), P[8 * g + i]), t0, t1);
-            f2_split(f2_mul(P[8 * g + i], P[8 * g + i]), n0, n1);
-            tn[i] = f2(__fadd_rn(t0, t1), __fadd_rn(n0, n1));
+            T[i] = f2_prod(T[i], P[8 * g + i], nz);
+            N[i] = f2_prod(P[8 * g + i], P[8 * g + i], nz);
         }
-#pragma unroll
-        for (int w = 8; w > 1; w >>= 1) {
-#pragma unroll
-            for (int i = 0; i < w / 2; ++i) tn[i] = f2_add(tn[2 * i], tn[2 * i + 1]);
-        }
-        float tg, ng;
-        f2_split(tn[0], tg, ng);
+        const float tg = pair_tree16(T), ng = pair_tree16(N);
         pq[g] = p;
         nq[g] = live ? ng : 0.0f;
         ptq[g] = live ? __fmul_rn(p, tg) : 0.0f;
@@ -231,12 +262,8 @@ __device__ __forceinline__ void sr_vector(const uint64_t (&P)[32], float g, floa
 #pragma unroll
     for (int gq = 0; gq < 4; ++gq) {
         float y[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f2_split(P[8 * gq + i], y[2 * i], y[2 * i + 1]);
-        const float m0 = absmax3(y[0], y[1], y[2]), m1 = absmax3(y[3], y[4], y[5]);
-        const float m2 = absmax3(y[6], y[7], y[8]), m3 = absmax3(y[9], y[10], y[11]);
-        const float m4 = absmax3(y[12], y[13], y[14]);
-        const float a = max2n(max3(m0, m1, m2), max3(m3, m4, fabsf(y[15])));
+        group_values(P, gq, y);
+        const float a = group_absmax(y);
         amax = max2n(amax, a);
         float q[16];
         if (zero_view || !(a >= kTiny)) {
@@ -318,7 +345,10 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     __shared__ __align__(8) uint64_t bar[NS];
     __shared__ uint32_t done_cnt[NS];           // warps done reading the stage, summed over its rounds
     __shared__ int last_issued[NS];             // local index of the last tile loaded into the stage
-    __shared__ __align__(16) uint2 sgn2[64];    // sign flips of elements 2n, 2n+1 at bit 31 of .x, .y
+    // sign flips (at bit 31) of elements 2n, 2n + 1, 2n + 8, 2n + 9 in .x, .y, .z, .w: the four
+    // elements of two pair registers (entries with bit 2 of n set are not used)
+    __shared__ __align__(16) uint4 sgn4[64];
+    __shared__ float s_nz;
 
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int team = warp >= Cfg::kTeamWarps ? 1 : 0;
@@ -358,10 +388,13 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     if (t < 64) {
         const uint4 sw = rotation_sign_words(seed);   // bit i of the 128 signs: element i negated
         const uint32_t w[4] = {sw.x, sw.y, sw.z, sw.w};
+        auto flip = [&](int e) { e &= 127; return ((w[e >> 5] >> (e & 31)) & 1u) << 31; };
         const int e = 2 * t;
-        sgn2[t] = make_uint2(((w[e >> 5] >> (e & 31)) & 1u) << 31, ((w[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) << 31);
+        sgn4[t] = make_uint4(flip(e), flip(e + 1), flip(e + 8), flip(e + 9));
     }
+    if (t == 0) s_nz = -0.0f;
     __syncthreads();
+    const uint64_t nz = neg_zero_pair(&s_nz);   // addend of f2_prod
     if (t == 0)
         for (int64_t i = 0; i < NS && i < my_tiles; ++i) issue(i);
 
@@ -389,16 +422,16 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         }
     }
     // forward view of the rows (kModeFwdRowEdenCol): tensor scale and the block's scale tables
-    __shared__ float tab_d[128], tab_r[128];
-    float g6_f = 0.0f, g4_f = 0.0f;
+    __shared__ float tab_d[128], tab_r[129];
+    Fwd46Consts kc_f{0.0f, 0.0f, 0.0f, 0.0f};
     if constexpr (MODE == kModeFwdRowEdenCol) {
         if (blockIdx.x == 0 && t == 0) check_finite_word(*row_amax);   // outputs then unspecified
         const float g = fwd46_tensor_scale(row_amax);
-        g6_f = __fmul_rn(g, 6.0f);
-        g4_f = __fmul_rn(g, 4.0f);
+        kc_f = fwd46_consts(g);
         if (blockIdx.x == 0 && t == 0) *out.row_g = g;
         fwd46_tables(g, tab_d, tab_r);
         __syncthreads();
+        kc_f.nz = neg_zero_pair(&tab_r[128]);
     }
     const float sigma = h ? -1.0f : 1.0f;
     const uint64_t sg = f2(sigma, sigma), nsg = f2(-sigma, -sigma);
@@ -406,12 +439,21 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
     const int u = (t & (Cfg::kTeamWarps * 32 - 1)) >> 1;   // the pair's row (or column) of the tile
     float amax = 0.0f;
     const int64_t i0 = kBoth ? 0 : team, step = kBoth ? 1 : 2;
-    for (int64_t i = i0; i < my_tiles; i += step) {
+    // tile coordinates (row, column of tiles), advanced without a division per tile
+    const int64_t adv = step * (int64_t)gridDim.x, adv_r = adv / tiles_c, adv_c = adv % tiles_c;
+    int64_t t_r = ((int64_t)blockIdx.x + i0 * (int64_t)gridDim.x) / tiles_c;
+    int64_t t_c = ((int64_t)blockIdx.x + i0 * (int64_t)gridDim.x) % tiles_c;
+    for (int i = (int)i0; i < (int)my_tiles; i += (int)step) {
+        const int64_t r0 = t_r << 7, c0 = t_c << 7;
+        t_c += adv_c;
+        t_r += adv_r;
+        if (t_c >= tiles_c) {
+            t_c -= tiles_c;
+            ++t_r;
+        }
         const int s = (int)(i % NS);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, (uint32_t)((i / NS) & 1)))) break;   // warp-uniform
         const uint8_t *tb = buf0 + s * Cfg::kTileBytes;
-        const int64_t tile = blockIdx.x + i * (int64_t)gridDim.x;
-        const int64_t r0 = (tile / tiles_c) << 7, c0 = (tile % tiles_c) << 7;
         uint64_t P[32];
         // A tile is two 128x64 boxes with the 128-byte swizzle: element (r, c) sits at byte
         // (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
@@ -428,7 +470,7 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
                     const uint4 a = lds128(rbase + ((uint32_t)((2 * gq) ^ (u & 7)) << 4));
                     const uint4 b = lds128(rbase + ((uint32_t)((2 * gq + 1) ^ (u & 7)) << 4));
                     const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                    scw |= fwd46_group(w, g6_f, g4_f, tab_d, tab_r, cw[2 * gq], cw[2 * gq + 1]) << (8 * gq);
+                    scw |= fwd46_group(w, kc_f, tab_d, tab_r, cw[2 * gq], cw[2 * gq + 1]) << (8 * gq);
                 }
                 release(s, i);
                 const int64_t vr = r0 + u;
@@ -440,48 +482,54 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             }
         }
         if (rows) {
-            // row u, elements [64h, 64h + 64); register chunk c holds element chunk 8h + (c ^ 4h),
-            // whose 16 bytes sit at swizzled chunk (c ^ 4h ^ (u % 8)) of row u in box h
+            // row u, elements [64h, 64h + 64) of the tile row (box h).  Slot group gq = a + 2b
+            // holds element chunks cl = 2a + 4b (low halves) and cl + 1 (high halves) of the
+            // thread's half, with thread 1's quarters swapped (cl ^ 4h); the swizzled 16 bytes of
+            // chunk c sit at chunk c ^ (u % 8) of row u.  Stride 1 is taken here.
             const uint32_t rbase = tbu + h * 16384 + u * 128, rx = (uint32_t)((4 * h) ^ (u & 7)) << 4;
-            const uint32_t sbase = smem_u32(&sgn2[0]) + 256 * h, sx = 128 * h;
+            const uint32_t sbase = smem_u32(&sgn4[0]) + 512 * h, sx = 256 * h;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = lds128(rbase + (rx ^ (uint32_t)(c << 4)));
-                const uint32_t sa = sbase + (sx ^ (uint32_t)(32 * c));
-                const uint4 m01 = lds128(sa), m23 = lds128(sa + 16);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const uint32_t ml[4] = {m01.x, m01.z, m23.x, m23.z}, mh[4] = {m01.y, m01.w, m23.y, m23.w};
+            for (int gq = 0; gq < 4; ++gq) {
+                const uint32_t cl = 2 * (gq & 1) + 4 * (gq >> 1);
+                const uint4 L = lds128(rbase + (rx ^ (cl << 4))), H = lds128(rbase + (rx ^ ((cl + 1) << 4)));
+                const uint32_t wl[4] = {L.x, L.y, L.z, L.w}, wh[4] = {H.x, H.y, H.z, H.w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float x0 = __uint_as_float((w[k] << 16) + ml[k]);   // adding 2^31 flips the sign bit
-                    const float x1 = __uint_as_float((w[k] & 0xFFFF0000u) ^ mh[k]);
-                    P[4 * c + k] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 m = lds128(sbase + (sx ^ (64 * cl + 16 * i)));
+                    // adding 2^31 flips the sign bit
+                    const uint64_t a = f2(__uint_as_float((wl[i] << 16) + m.x), __uint_as_float((wh[i] << 16) + m.z));
+                    const uint64_t b = f2(__uint_as_float((wl[i] & 0xFFFF0000u) ^ m.y),
+                                          __uint_as_float((wh[i] & 0xFFFF0000u) ^ m.w));
+                    P[8 * gq + 2 * i] = f2_add(a, b);
+                    P[8 * gq + 2 * i + 1] = f2_sub(a, b);
                 }
             }
         } else {
-            // column u, rows [64h, 64h + 64); slot j holds rows 2n, 2n + 1 of the half with
-            // n = (j + 16h) % 32, i.e. tile rows 96h + 2j (j < 16) and 32h + 2j (j >= 16).  The
-            // swizzle term depends on the row only through (2j + d) % 8, a constant per load.
+            // column u, rows [64h, 64h + 64) of the tile.  Slot 16b + 8a + j holds rows
+            // R0 + 16a + j and R0 + 16a + j + 8 with R0 = 64h + 32(b ^ h) (thread 1's quarters
+            // swapped).  R0 is a multiple of 32, so the swizzle term of row R0 + r depends only
+            // on r % 8: one base address per value of r % 8 and half b.  Stride 1 is taken here.
             const uint32_t colbase = (uint32_t)((u >> 6) * 16384 + (u & 7) * 2 + (((u & 63) >> 3) << 4));
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const uint32_t hb = tbu + (half == 0 ? 12288u : 4096u) * h;
-                const uint32_t sb = smem_u32(&sgn2[0]) + (half == 0 ? 384u : 128u) * h;
+                const uint32_t hb = tbu + (half == 0 ? 12288u * h : 4096u + 4096u * h);
+                const uint32_t sb = smem_u32(&sgn4[0]) + 512 * h + (half == 0 ? 256u * h : 256u - 256u * h);
                 uint32_t X[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) X[k] = hb + (colbase ^ (uint32_t)(k << 4));
 #pragma unroll
-                for (int jj = 0; jj < 16; jj += 2) {
-                    const int j = 16 * half + jj;
-                    const uint4 m = lds128(sb + 8 * j);
-                    const uint32_t u0 = lds16(X[(2 * j) & 7] + 256 * j);
-                    const uint32_t u1 = lds16(X[(2 * j + 1) & 7] + 256 * j + 128);
-                    const uint32_t u2 = lds16(X[(2 * j + 2) & 7] + 256 * j + 256);
-                    const uint32_t u3 = lds16(X[(2 * j + 3) & 7] + 256 * j + 384);
-                    const float x0 = __uint_as_float((u0 << 16) + m.x), x1 = __uint_as_float((u1 << 16) + m.y);
-                    const float x2 = __uint_as_float((u2 << 16) + m.z), x3 = __uint_as_float((u3 << 16) + m.w);
-                    P[j] = f2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
-                    P[j + 1] = f2(__fadd_rn(x2, x3), __fsub_rn(x2, x3));
+                for (int a = 0; a < 2; ++a) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int j = 2 * i, r = 16 * a + j;
+                        const uint4 m = lds128(sb + 16 * i + 128 * a);
+                        const uint32_t u0 = lds16(X[j] + 128 * r), u1 = lds16(X[j + 1] + 128 * (r + 1));
+                        const uint32_t u2 = lds16(X[j] + 128 * (r + 8)), u3 = lds16(X[j + 1] + 128 * (r + 9));
+                        const uint64_t va = f2(__uint_as_float((u0 << 16) + m.x), __uint_as_float((u2 << 16) + m.z));
+                        const uint64_t vb = f2(__uint_as_float((u1 << 16) + m.y), __uint_as_float((u3 << 16) + m.w));
+                        P[16 * half + 8 * a + j] = f2_add(va, vb);
+                        P[16 * half + 8 * a + j + 1] = f2_sub(va, vb);
+                    }
                 }
             }
         }
@@ -493,12 +541,12 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
         if constexpr (MODE == kModeEden) {
             uint32_t cw[8];
             float Pq[4];
-            msed_vector(P, sg, nsg, cw, Pq, amax);
+            msed_vector(P, sg, nsg, nz, cw, Pq, amax);
             msed_store(vcodes, rows ? row_P : col_P, vr, b0 >> 4, VC, h, cw, Pq);
         } else if constexpr (MODE == kModeFwdRowEdenCol) {   // column warps (rows returned above)
             uint32_t cw[8];
             float Pq[4];
-            msed_vector(P, sg, nsg, cw, Pq, amax);
+            msed_vector(P, sg, nsg, nz, cw, Pq, amax);
             msed_store(vcodes, col_P, vr, b0 >> 4, VC, h, cw, Pq);
         } else if constexpr (MODE == kModeMax) {
             rotate_tail(P, sg, nsg);

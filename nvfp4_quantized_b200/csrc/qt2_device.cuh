@@ -52,21 +52,19 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
     return r;
 }
 
-// Two E2M1 codes in the low byte of `byte` -> f16x2 (low nibble -> low half).
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "r"(byte));
-    return h2;
-}
-
-// Eight packed E2M1 codes -> their exact values as fp32 (nibble i -> out[i]).
-__device__ __forceinline__ void e2m1x8_values(uint32_t codes, float (&out)[8]) {
+// Sixteen E2M1 codes (c0: elements 0..7, c1: elements 8..15, element i in nibble i % 8) -> their
+// exact values as fp32 pairs V[i] = (value of element i, value of element i + 8).
+__device__ __forceinline__ void e2m1x16_pairs(uint32_t c0, uint32_t c1, uint64_t (&V)[8]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t h = e2m1x2_to_f16x2(codes >> (8 * i));
-        asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-            : "=f"(out[2 * i]), "=f"(out[2 * i + 1])
-            : "r"(h));
+    for (int j = 0; j < 4; ++j) {
+        asm("{\n\t.reg .b8 p, q;\n\t.reg .b32 hp, hq;\n\t.reg .f16 p0, p1, q0, q1;\n\t.reg .f32 a, b, c, d;\n\t"
+            "cvt.u8.u32 p, %2;\n\tcvt.u8.u32 q, %3;\n\t"
+            "cvt.rn.f16x2.e2m1x2 hp, p;\n\tcvt.rn.f16x2.e2m1x2 hq, q;\n\t"
+            "mov.b32 {p0, p1}, hp;\n\tmov.b32 {q0, q1}, hq;\n\t"
+            "cvt.f32.f16 a, p0;\n\tcvt.f32.f16 b, q0;\n\tcvt.f32.f16 c, p1;\n\tcvt.f32.f16 d, q1;\n\t"
+            "mov.b64 %0, {a, b};\n\tmov.b64 %1, {c, d};\n\t}"
+            : "=l"(V[2 * j]), "=l"(V[2 * j + 1])
+            : "r"(c0 >> (8 * j)), "r"(c1 >> (8 * j)));
     }
 }
 

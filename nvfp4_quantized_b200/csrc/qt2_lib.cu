@@ -139,6 +139,25 @@ __global__ void selftest_wait_kernel() {
     if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0);
 }
 
+// Self-test of the quantizers' division shortcuts: for every binary32 value x whose biased
+// exponent lies in [e_lo, e_hi] (every significand), rcp_rn(x) against the IEEE reciprocal
+// (counted in mismatches[0]) and div6_rn(x) against the IEEE quotient x/6 (mismatches[1]).
+__global__ void selftest_division_kernel(uint32_t e_lo, uint32_t e_hi, unsigned long long *mismatches) {
+    const uint64_t n = (uint64_t)(e_hi - e_lo + 1) << 23;
+    unsigned bad_r = 0, bad_d = 0;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x) {
+        const float x = __uint_as_float((uint32_t)(((uint64_t)e_lo << 23) + i));
+        bad_r += __float_as_uint(rcp_rn(x)) != __float_as_uint(__frcp_rn(x));
+        bad_d += __float_as_uint(div6_rn(x)) != __float_as_uint(__fdiv_rn(x, 6.0f));
+    }
+    bad_r = __reduce_add_sync(0xFFFFFFFFu, bad_r);
+    bad_d = __reduce_add_sync(0xFFFFFFFFu, bad_d);
+    if ((threadIdx.x & 31) == 0) {
+        if (bad_r) atomicAdd(&mismatches[0], (unsigned long long)bad_r);
+        if (bad_d) atomicAdd(&mismatches[1], (unsigned long long)bad_d);
+    }
+}
+
 cudaError_t launch_fwd46_local(const uint16_t *x, int64_t R, int64_t C, int64_t ld, DevView out, cudaStream_t s) {
     QT2_LAUNCH_SITE();
     fwd46_local_kernel<<<(unsigned)(R / 128 * kLocalCluster), kLocalThreads, 0, s>>>(x, R, C, ld, out.codes,
@@ -825,6 +844,21 @@ qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream) {
     if (fa == kFaultFail) return QT2_ERR_CUDA;
     if (fa == kFaultSkip) return QT2_OK;
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return from_cuda(cudaGetLastError());
+}
+
+qt2_status qt2_selftest_division(uint32_t exp_lo, uint32_t exp_hi, unsigned long long *mismatches,
+                                  qt2_stream_t stream) {
+    QT2_TRACE();
+    if (!mismatches || exp_lo < 1 || exp_hi > 254 || exp_lo > exp_hi) return QT2_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mismatches) & 7u) != 0) return QT2_ERR_ALIGN;
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    const int fa = fault_at("launch");
+    if (fa == kFaultFail) return QT2_ERR_CUDA;
+    if (fa == kFaultSkip) return QT2_OK;
+    selftest_division_kernel<<<(unsigned)sm_count() * 8, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        exp_lo, exp_hi, mismatches);
     return from_cuda(cudaGetLastError());
 }
 

@@ -98,6 +98,43 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// RN(a*b) on both halves as a fused multiply-add with addend nz = (-0, -0) (exact: adding -0
+// changes no rounded product and keeps the sign of a zero one).  A product that feeds an
+// addition or a subtraction is formed this way: a packed multiply followed by a packed add can
+// be contracted into one fused multiply-add by the code generator, which would skip the
+// product's rounding.  nz must be a run-time value (read from shared memory, see neg_zero_pair):
+// with a constant -0 addend the FMA could be rewritten as a plain multiply and contracted again.
+__device__ __forceinline__ uint64_t f2_prod(uint64_t a, uint64_t b, uint64_t nz) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(nz));
+    return r;
+}
+// (-0, -0) from a shared word that the block's first thread set to -0 before a barrier.
+__device__ __forceinline__ uint64_t neg_zero_pair(const float *word) {
+    const float z = *reinterpret_cast<const volatile float *>(word);
+    return f2(z, z);
+}
+
+// Balanced tree of 16 values held as 8 pairs (element i, element i + 8): levels 1..3 pair
+// adjacent registers on both halves at once, level 4 adds the halves -- the same tree as the
+// plain one over elements 0..15 ((0+1)+(2+3))+... .
+__device__ __forceinline__ float pair_tree16(uint64_t (&T)[8]) {
+#pragma unroll
+    for (int w = 8; w > 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w / 2; ++i) T[i] = f2_add(T[2 * i], T[2 * i + 1]);
+    }
+    float lo, hi;
+    f2_split(T[0], lo, hi);
+    return __fadd_rn(lo, hi);
+}
+
+// max |x| over three values; exact, so the grouping of a max tree does not matter
+__device__ __forceinline__ float absmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
 
 // ---------------------------------------------------------------------------------------------
 // Forward quantizer, row view: RTN onto E2M1 with the 4/6 grid choice per 1x16 group
@@ -105,57 +142,84 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // One thread per 16-element group; a warp covers 32 consecutive groups of one row.
 // Candidate k (6 or 4): s = RNE_E4M3(a/(g*k)), d = s*g, codes = RNE_E2M1(x*(1/d)),
 // err = tree sum of (x - val*d)^2; a zero scale gives sign-preserving zero codes (x*0) and
-// err = sum x^2.  Keep 4 iff err4 < err6.  Elements 2j, 2j+1 share a packed register; the two
-// candidates' trees run side by side from level 2 on.
+// err = sum x^2.  Keep 4 iff err4 < err6.  A packed register holds elements i and i + 8 of the
+// group, so every step but the last tree level runs on f32x2 instructions.
 // ---------------------------------------------------------------------------------------------
 struct Fwd46Scale {
     uint32_t code;
-    float d;
+    uint64_t dd;       // (d, d)
     uint64_t rr;       // (1/d, 1/d)
 };
 
-// d and 1/d depend on the scale code only (g is fixed per tensor): the block tabulates them once
-// for the 128 non-negative E4M3 codes (tab_d[c] = RN(val(c)*g), tab_r[c] = RN(1/tab_d[c]),
-// tab_r[0] = 0), so a candidate costs one division, one convert and two shared loads.
-__device__ __forceinline__ Fwd46Scale fwd46_scale(float a, float gk, const float *tab_d, const float *tab_r) {
-    Fwd46Scale c;
-    c.code = e4m3_rne(__fdiv_rn(a, gk));
-    const float r = tab_r[c.code];
-    c.rr = f2(r, r);
-    c.d = tab_d[c.code];
+// Per-tensor constants: g*6, g*4 and their reciprocals RN(1/(g*k)).
+struct Fwd46Consts {
+    float g6, g4, i6, i4;
+    uint64_t nz;   // (-0, -0) read from shared memory (f2_prod), set after the tables
+};
+__device__ __forceinline__ Fwd46Consts fwd46_consts(float g) {
+    Fwd46Consts c;
+    c.g6 = __fmul_rn(g, 6.0f);
+    c.g4 = __fmul_rn(g, 4.0f);
+    c.i6 = __frcp_rn(c.g6);
+    c.i4 = __frcp_rn(c.g4);
+    c.nz = 0;
     return c;
 }
 
-// Codes of one candidate (two words: elements 0..7, 8..15) and its 8 level-1 error sums
-// (element pairs 2j, 2j+1).
-__device__ __forceinline__ void fwd46_candidate(const uint64_t (&X)[8], const Fwd46Scale &sc, uint32_t (&codes)[2],
-                                                float (&e1)[8]) {
+// RNE_E4M3(RN(a / gk)) from t' = RN(a * RN(1/gk)): t' is within 3 ulps of RN(a/gk) (two
+// roundings of relative size 2^-24 each, against an ulp of at least 2^-24 of the value), so
+// when t' lies in the E4M3 normal range and its 20 bits below the E4M3 mantissa are more than 3
+// ulps from the rounding midpoint 0x80000, RN(a/gk) rounds to the same E4M3 value; otherwise
+// (near a midpoint, or in the subnormal range below 2^-6) the quotient is formed exactly.
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float a, float gk, float inv_gk) {
+    const float tp = __fmul_rn(a, inv_gk);
+    const uint32_t low = __float_as_uint(tp) & 0xFFFFFu;
+    const bool safe = tp >= 0x1p-6f && (low < 0x80000u - 3u || low > 0x80000u + 3u);
+    return e4m3_rne(safe ? tp : __fdiv_rn(a, gk));
+}
+
+// d and 1/d depend on the scale code only (g is fixed per tensor): the block tabulates them once
+// for the 128 non-negative E4M3 codes (tab_d[c] = RN(val(c)*g), tab_r[c] = RN(1/tab_d[c]),
+// tab_r[0] = 0), so a candidate costs a multiply, a convert and two shared loads.
+__device__ __forceinline__ Fwd46Scale fwd46_scale(float a, float gk, float inv_gk, const float *tab_d,
+                                                  const float *tab_r) {
+    Fwd46Scale c;
+    c.code = e4m3_of_quotient(a, gk, inv_gk);
+    const float r = tab_r[c.code], d = tab_d[c.code];
+    c.rr = f2(r, r);
+    c.dd = f2(d, d);
+    return c;
+}
+
+// Codes of one candidate (two words: elements 0..7, 8..15) and its squared errors as pairs
+// (element i, element i + 8).  X[i] = (x_i, x_{i+8}).
+__device__ __forceinline__ void fwd46_candidate(const uint64_t (&X)[8], const Fwd46Scale &sc, uint64_t nz,
+                                                uint32_t (&codes)[2], uint64_t (&E)[8]) {
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f2_split(f2_mul(X[i], sc.rr), q[i], q[i + 8]);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        float q[8];
+        float qh[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) f2_split(f2_mul(X[4 * h + i], sc.rr), q[2 * i], q[2 * i + 1]);
-        codes[h] = e2m1x8(q);
-        float val[8];
-        e2m1x8_values(codes[h], val);
+        for (int i = 0; i < 8; ++i) qh[i] = q[8 * h + i];
+        codes[h] = e2m1x8(qh);
+    }
+    // x - val*d and the squares, each product rounded on its own (f2_prod)
+    uint64_t V[8];
+    e2m1x16_pairs(codes[0], codes[1], V);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            // x - val*d in scalar mul.rn/sub.rn, which are never fused: a packed multiply feeding a
-            // packed subtract may be contracted into one fused multiply-add
-            float x0, x1;
-            f2_split(X[4 * h + i], x0, x1);
-            const float e0 = __fsub_rn(x0, __fmul_rn(val[2 * i], sc.d));
-            const float e1v = __fsub_rn(x1, __fmul_rn(val[2 * i + 1], sc.d));
-            float s0, s1;
-            f2_split(f2_mul(f2(e0, e1v), f2(e0, e1v)), s0, s1);
-            e1[4 * h + i] = __fadd_rn(s0, s1);
-        }
+    for (int i = 0; i < 8; ++i) {
+        const uint64_t e = f2_sub(X[i], f2_prod(V[i], sc.dd, nz));
+        E[i] = f2_prod(e, e, nz);
     }
 }
 
 // The block's tables of d = RN(val(c) * g) and RN(1/d) for the 128 non-negative E4M3 codes c
-// (tab_r[0] = 0); called by the first 128 threads, followed by a barrier.
+// (tab_r[0] = 0), and tab_r[128] = -0 (the addend of f2_prod); called by every thread, followed
+// by a barrier.  tab_r has 129 entries.
 __device__ __forceinline__ void fwd46_tables(float g, float *tab_d, float *tab_r) {
+    if (threadIdx.x == 0) tab_r[128] = -0.0f;
     if (threadIdx.x < 128) {
         const float d = __fmul_rn(e4m3_value(threadIdx.x), g);
         tab_d[threadIdx.x] = d;
@@ -163,39 +227,39 @@ __device__ __forceinline__ void fwd46_tables(float g, float *tab_d, float *tab_r
     }
 }
 
-// One 16-element group (8 words of bf16 pairs, element 2i in the low half of word i): its two
-// code words and its scale code.
-__device__ __forceinline__ uint32_t fwd46_group(const uint32_t (&w)[8], float g6, float g4, const float *tab_d,
-                                                const float *tab_r, uint32_t &code0, uint32_t &code1) {
-    uint64_t X[8];
-    float m8[8];
+// Pair registers (x_i, x_{i+8}) and max |x| of one 16-element group given as 8 words of bf16
+// pairs (element 2i in the low half of word i).
+__device__ __forceinline__ float fwd46_unpack(const uint32_t (&w)[8], uint64_t (&X)[8]) {
+    float x[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-        X[i] = f2(lo, hi);
-        m8[i] = fmaxf(fabsf(lo), fabsf(hi));
+        x[2 * i] = bf16_lo(w[i]);
+        x[2 * i + 1] = bf16_hi(w[i]);
     }
 #pragma unroll
-    for (int s = 8; s > 1; s >>= 1) {
-#pragma unroll
-        for (int i = 0; i < s / 2; ++i) m8[i] = fmaxf(m8[2 * i], m8[2 * i + 1]);
-    }
-    const float a = m8[0];
-    const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
+    for (int i = 0; i < 8; ++i) X[i] = f2(x[i], x[i + 8]);
+    const float m0 = absmax3f(x[0], x[1], x[2]), m1 = absmax3f(x[3], x[4], x[5]);
+    const float m2 = absmax3f(x[6], x[7], x[8]), m3 = absmax3f(x[9], x[10], x[11]);
+    const float m4 = absmax3f(x[12], x[13], x[14]);
+    float a;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(a) : "f"(m0), "f"(m1), "f"(m2));
+    float b;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(b) : "f"(m3), "f"(m4), "f"(fabsf(x[15])));
+    return fmaxf(a, b);
+}
+
+// One 16-element group (8 words of bf16 pairs, element 2i in the low half of word i): its two
+// code words and its scale code.
+__device__ __forceinline__ uint32_t fwd46_group(const uint32_t (&w)[8], const Fwd46Consts &k, const float *tab_d,
+                                                const float *tab_r, uint32_t &code0, uint32_t &code1) {
+    uint64_t X[8];
+    const float a = fwd46_unpack(w, X);
+    const Fwd46Scale s6 = fwd46_scale(a, k.g6, k.i6, tab_d, tab_r), s4 = fwd46_scale(a, k.g4, k.i4, tab_d, tab_r);
     uint32_t c6[2], c4[2];
-    float e6[8], e4[8];
-    fwd46_candidate(X, s6, c6, e6);
-    fwd46_candidate(X, s4, c4, e4);
-    uint64_t t[8];   // (candidate 6, candidate 4) level-1 sums, then levels 2..4 together
-#pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
-#pragma unroll
-    for (int s = 8; s > 1; s >>= 1) {
-#pragma unroll
-        for (int i = 0; i < s / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
-    }
-    float err6, err4;
-    f2_split(t[0], err6, err4);
+    uint64_t e6[8], e4[8];
+    fwd46_candidate(X, s6, k.nz, c6, e6);
+    fwd46_candidate(X, s4, k.nz, c4, e4);
+    const float err6 = pair_tree16(e6), err4 = pair_tree16(e4);
     const bool pick4 = err4 < err6;                    // a tie keeps the full grid
     code0 = pick4 ? c4[0] : c6[0];
     code1 = pick4 ? c4[1] : c6[1];
@@ -285,29 +349,55 @@ __global__ void __launch_bounds__(256) fwd46_coop_kernel(const uint16_t *__restr
     }
     const float A = __uint_as_float(abits);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
-    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    Fwd46Consts kc = fwd46_consts(g);
     if (blockIdx.x == 0 && threadIdx.x == 0) *tensor_scale = g;
-    __shared__ float tab_d[128], tab_r[128];
+    __shared__ float tab_d[128], tab_r[129];
     fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
+    kc.nz = neg_zero_pair(&tab_r[128]);
+    // group gi = r * G + q; the grid-stride step advances (r, q) without a division, and the
+    // next group's 32 bytes are loaded before the current one is quantized
     const uint32_t G = (uint32_t)(C >> 4);
-    const uint64_t total = (uint64_t)R * G;
-    const bool small = total <= 0xFFFFFFFFull;
-    for (uint64_t gi = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < total;
-         gi += (uint64_t)gridDim.x * blockDim.x) {
-        const uint64_t r = small ? (uint64_t)((uint32_t)gi / G) : gi / G;
-        const uint32_t q = (uint32_t)(gi - r * G);
+    const uint64_t total = (uint64_t)R * G, stride = (uint64_t)gridDim.x * blockDim.x;
+    const uint64_t step_r = stride / G;
+    const uint32_t step_q = (uint32_t)(stride % G);
+    uint64_t gi = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint64_t r = gi / G;
+    uint32_t q = (uint32_t)(gi % G);
+    uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
+    if (gi < total) {
         const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (uint64_t)q * 16);
-        const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
+        w0 = __ldcs(src);
+        w1 = __ldcs(src + 1);
+    }
+    while (gi < total) {   // warp-uniform: a warp's 32 groups are consecutive and total % 32 == 0
+        const uint64_t gn = gi + stride;
+        uint64_t rn = r + step_r;
+        uint32_t qn = q + step_q;
+        if (qn >= G) {
+            qn -= G;
+            ++rn;
+        }
+        uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+        if (gn < total) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + rn * ld + (uint64_t)qn * 16);
+            n0 = __ldcs(src);
+            n1 = __ldcs(src + 1);
+        }
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t code0, code1;
-        const uint32_t sc = fwd46_group(w, g6, g4, tab_d, tab_r, code0, code1);
+        const uint32_t sc = fwd46_group(w, kc, tab_d, tab_r, code0, code1);
         *reinterpret_cast<uint2 *>(codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8) = make_uint2(code0, code1);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if ((lane & 3) == 0)
             *reinterpret_cast<uint32_t *>(scales + sf_offset((int64_t)r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        gi = gn;
+        r = rn;
+        q = qn;
+        w0 = n0;
+        w1 = n1;
     }
 }
 
@@ -368,28 +458,36 @@ __global__ void __cluster_dims__(kLocalCluster, 1, 1) __launch_bounds__(kLocalTh
     }
     const float A = __uint_as_float(bmax);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
-    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    Fwd46Consts kc = fwd46_consts(g);
     if (rank == 0 && threadIdx.x == 0) g_blocks[blk] = g;
-    __shared__ float tab_d[128], tab_r[128];
+    __shared__ float tab_d[128], tab_r[129];
     fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
+    kc.nz = neg_zero_pair(&tab_r[128]);
     // the CTA's groups, one per thread and round (4 consecutive lanes: one scale word)
     const uint32_t G = (uint32_t)(C >> 4);
     const uint32_t total = 32u * G;                    // a multiple of 256
+    const uint32_t step_r = kLocalThreads / G, step_q = kLocalThreads % G;
+    uint32_t rr = threadIdx.x / G, q = threadIdx.x % G;   // (row within the CTA's 32, group)
     for (uint32_t gi = threadIdx.x; gi < total; gi += kLocalThreads) {
-        const int64_t r = r0 + gi / G;
-        const uint32_t q = gi % G;
+        const int64_t r = r0 + rr;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + r * ld + (int64_t)q * 16);
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t code0, code1;
-        const uint32_t sc = fwd46_group(w, g6, g4, tab_d, tab_r, code0, code1);
+        const uint32_t sc = fwd46_group(w, kc, tab_d, tab_r, code0, code1);
         *reinterpret_cast<uint2 *>(codes + r * (C >> 1) + (int64_t)q * 8) = make_uint2(code0, code1);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
         if ((lane & 3) == 0)
             *reinterpret_cast<uint32_t *>(scales + sf_offset(r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        rr += step_r;
+        q += step_q;
+        if (q >= G) {
+            q -= G;
+            ++rr;
+        }
     }
 }
 
@@ -419,14 +517,15 @@ __global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restric
         return;
     }
     const float g = fwd46_tensor_scale(amax_word);
-    const float g6 = __fmul_rn(g, 6.0f), g4 = __fmul_rn(g, 4.0f);
+    Fwd46Consts kc = fwd46_consts(g);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         *row_g = g;
         *col_g = g;
     }
-    __shared__ float tab_d[128], tab_r[128];
+    __shared__ float tab_d[128], tab_r[129];
     fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
+    kc.nz = neg_zero_pair(&tab_r[128]);
 
     const int lane = threadIdx.x & 31, j = lane & 15;
     const int64_t QB = C >> 4;                              // blocks along C (even)
@@ -440,29 +539,17 @@ __global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restric
         const uint4 w0 = __ldcs(src), w1 = __ldcs(src + 1);
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint64_t X[8];
-        float a = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
-            X[i] = f2(lo, hi);
-            a = fmaxf(a, fmaxf(fabsf(lo), fabsf(hi)));
-        }
+        float a = fwd46_unpack(w, X);
 #pragma unroll
         for (int m = 1; m < 16; m <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, m));   // block max (exact)
-        const Fwd46Scale s6 = fwd46_scale(a, g6, tab_d, tab_r), s4 = fwd46_scale(a, g4, tab_d, tab_r);
+        const Fwd46Scale s6 = fwd46_scale(a, kc.g6, kc.i6, tab_d, tab_r);
+        const Fwd46Scale s4 = fwd46_scale(a, kc.g4, kc.i4, tab_d, tab_r);
         uint32_t c6[2], c4[2];
-        float e6[8], e4[8];
-        fwd46_candidate(X, s6, c6, e6);
-        fwd46_candidate(X, s4, c4, e4);
-        uint64_t t[8];   // (candidate 6, candidate 4): the row's tree, then the rows' tree
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = f2(e6[i], e4[i]);
-#pragma unroll
-        for (int sz = 8; sz > 1; sz >>= 1) {
-#pragma unroll
-            for (int i = 0; i < sz / 2; ++i) t[i] = f2_add(t[2 * i], t[2 * i + 1]);
-        }
-        uint64_t tb = t[0];
+        uint64_t e6[8], e4[8];
+        fwd46_candidate(X, s6, kc.nz, c6, e6);
+        fwd46_candidate(X, s4, kc.nz, c4, e4);
+        // (candidate 6, candidate 4): the row's tree, then the rows' tree
+        uint64_t tb = f2(pair_tree16(e6), pair_tree16(e4));
 #pragma unroll
         for (int m = 1; m < 16; m <<= 1) tb = f2_add(tb, shfl_xor_u64(tb, m));   // addition commutes: same bits
         float err6, err4;

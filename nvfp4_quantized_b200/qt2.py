@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
                 "qt2_quant_fwd46_local": (i32, [vp, i64, i64, i64, pv, vp]),
                 "qt2_selftest_wait_timeout": (i32, [vp]),
                 "qt2_set_fault_hook": (None, [FaultHookC, vp]),
+                "qt2_selftest_division": (i32, [u32, u32, vp, vp]),
                 "qt2_gemm_nvfp4_local": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
@@ -350,6 +351,15 @@ class fault_hook:
     def __exit__(self, *exc):
         lib().qt2_set_fault_hook(FaultHookC(), None)
         return False
+
+
+def qt2_selftest_division(exp_lo: int, exp_hi: int, stream=None) -> tuple[int, int]:
+    """(reciprocal, division by 6) mismatches of the kernels' forms against IEEE binary32 over
+    every value with biased exponent in [exp_lo, exp_hi] (synchronizes)."""
+    cnt = torch.zeros(2, dtype=torch.int64, device="cuda")
+    _check("qt2_selftest_division", lib().qt2_selftest_division(exp_lo, exp_hi, cnt.data_ptr(), _stream(stream)))
+    r, d = cnt.tolist()
+    return int(r), int(d)
 
 
 def qt2_selftest_wait_timeout(stream=None) -> None:

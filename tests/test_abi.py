@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 25
+    assert len(names) == 26
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
