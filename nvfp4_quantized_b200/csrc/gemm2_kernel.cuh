@@ -20,17 +20,18 @@
 //
 // Roles, per CTA of 384 threads (12 warps), persistent over 256x256 tiles (K = 256 per stage):
 //   warp 0             : producer.  Per stage, after "empty" (the MMAs that read the slot
-//                        completed), one lane loads the slot's own 128 rows of A, own 128 of the
-//                        256 B rows, the A scales of its rows and the B scales of all 256 rows
-//                        (each SM's tensor memory needs the scales of every B column): 38 KB,
-//                        reported to the leader's "full" barrier (the leader expects both SMs'
-//                        bytes).
-//   warp 2, leader     : scale copier.  After "full", copies the stage's 12 scale atoms from
+//                        completed), one lane loads the stage's scales -- A scales of its own
+//                        rows, B scales of all 256 rows (each SM's tensor memory needs the scales
+//                        of every B column) -- reported to the leader's "sfull" barrier, then its
+//                        own 128 rows of A and own 128 of the 256 B rows, reported to "full"
+//                        (the leader expects both SMs' bytes on each): 38 KB a stage.
+//   warp 2, leader     : scale copier.  After "sfull", copies the stage's 12 scale atoms from
 //                        both SMs' shared memory into their tensor memory (tcgen05.cp 32x128b,
 //                        replicated into the four lane quadrants, the layout the block-scaled
-//                        MMA reads) and commits to "sftm".  The stage's scale region is free by
-//                        then: its data could only land after the MMAs of the stage that last
-//                        used the region completed.
+//                        MMA reads) and commits to "sftm" -- while the stage's codes are still
+//                        in flight.  The stage's scale region is free by then: its data could
+//                        only land after the MMAs of the stage that last used the region
+//                        completed.
 //   warp 1             : allocates/frees 512 TMEM columns (both SMs); on the leader, after
 //                        "full" and "sftm", issues the four 256x256x64 MMAs of the stage and a
 //                        tcgen05.commit that frees the slot on both SMs ("empty").
@@ -163,9 +164,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     constexpr int S = Cfg::kStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    // barriers: full[S] sftm[S] empty[S] acc_full acc_empty
+    // barriers: full[S] sftm[S] empty[S] acc_full acc_empty sfull[S]
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + S * Cfg::kStageBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * S + 2);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * S + 2);
 
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -177,10 +178,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     const int total = my_tiles * nks;   // stages this pair runs
     const uint32_t full0 = smem_u32(bars), sftm0 = smem_u32(bars + S), empty0 = smem_u32(bars + 2 * S);
     const uint32_t acc_full = smem_u32(bars + 3 * S), acc_empty = acc_full + 8;
+    const uint32_t sfull0 = smem_u32(bars + 3 * S + 2);   // the stage's scale atoms landed
+
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8 * s, 1);    // the leader's producer (expects both SMs' bytes)
+            mbar_init(full0 + 8 * s, 1);    // codes: the leader's producer (expects both SMs' bytes)
+            mbar_init(sfull0 + 8 * s, 1);   // scale atoms: likewise
             mbar_init(sftm0 + 8 * s, 1);    // the scale copier's commit
             mbar_init(empty0 + 8 * s, 1);   // the MMA issuer's commit
         }
@@ -225,11 +229,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             const uint32_t st = smem_u32(base + s * Cfg::kStageBytes);
             const uint32_t fb = full_leader0 + 8 * s;
             if (elect_one()) {
-                if (leader) mbar_arrive_expect_tx(full0 + 8 * s, 2 * Cfg::kStageBytes);
+                // the scale atoms first, on their own barrier: the copier moves them into tensor
+                // memory while the codes are still in flight
+                const uint32_t sb = mapa_shared(sfull0, 0) + 8 * s;
+                if (leader) {
+                    mbar_arrive_expect_tx(sfull0 + 8 * s, 2 * (Cfg::kSfa + Cfg::kSfb));
+                    mbar_arrive_expect_tx(full0 + 8 * s, 2 * (Cfg::kA + Cfg::kB));
+                }
+                tma_load_2d_pair(st + Cfg::kA + Cfg::kB, &tmSFA, ks * 256, pm * 2 + (int)rank, sb);
+                tma_load_2d_pair(st + Cfg::kA + Cfg::kB + Cfg::kSfa, &tmSFB, ks * 256, pn * 2, sb);
                 tma_load_2d_pair(st, &tmA, ks * 128, pm * 256 + (int)rank * 128, fb);
                 tma_load_2d_pair(st + Cfg::kA, &tmB, ks * 128, pn * 256 + (int)rank * 128, fb);
-                tma_load_2d_pair(st + Cfg::kA + Cfg::kB, &tmSFA, ks * 256, pm * 2 + (int)rank, fb);
-                tma_load_2d_pair(st + Cfg::kA + Cfg::kB + Cfg::kSfa, &tmSFB, ks * 256, pn * 2, fb);
             }
             __syncwarp();
             issued = it + 1;
@@ -278,7 +288,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         // The stage's data landed, so the MMAs that last used its scale region completed.
         for (int j = 0; j < total; ++j) {
             const int s = j % S;
-            if (!mbar_wait_warp(full0 + 8 * s, (j / S) & 1)) break;
+            if (!mbar_wait_warp(sfull0 + 8 * s, (j / S) & 1)) break;
             tc_fence_after();
             const int nk = min(4, nkb - (j % nks) * 4);
             const uint32_t sfa = smem_u32(base + s * Cfg::kStageBytes + Cfg::kA + Cfg::kB), sfb = sfa + Cfg::kSfa;
@@ -374,7 +384,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         // both SMs' loads of a stage complete on the leader's barrier
         const int peer = (int)ld_shared_cluster_u32(mapa_shared(smem_u32(&issued_here), 1));
         const int last = max(issued, peer);
-        for (int it = consumed; it < last; ++it) mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
+        for (int it = consumed; it < last; ++it) {
+            mbar_wait(full0 + 8 * (it % S), (it / S) & 1);
+            mbar_wait(sfull0 + 8 * (it % S), (it / S) & 1);
+        }
     }
     if (leader && warp == 1 && lane == 0 && mma_done > 0) {
         const int it = mma_done - 1;

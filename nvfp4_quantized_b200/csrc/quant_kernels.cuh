@@ -609,12 +609,26 @@ __global__ void __launch_bounds__(256) msed_finalize_kernel(FinalizeJob j0, Fina
     if (bid == 0 && threadIdx.x == 0) *jb.tensor_scale = g;
     const int64_t words = (jb.VR * jb.VC) >> 6;
     const int64_t atoms_per_rowblock = jb.VC >> 6;
-    for (int64_t w = bid * blockDim.x + threadIdx.x; w < words; w += nb * blockDim.x) {
-        const int64_t atom = w >> 7, wi = w & 127;
-        const int64_t r = (atom / atoms_per_rowblock) * 128 + (wi & 3) * 32 + (wi >> 2);
-        const int64_t j4 = atom % atoms_per_rowblock;        // groups 4*j4 .. 4*j4+3 of view row r
-        const float4 p = __ldcs(jb.P + w);
+    // word w = atom * 128 + wi: the stride is a multiple of 128 words, so wi (the thread's row
+    // within the atom) is fixed and the atom's (row block, group quad) advance without a division;
+    // the next word is loaded before the current one is rounded
+    const int64_t stride = nb * (int64_t)blockDim.x;
+    const int64_t w0 = bid * (int64_t)blockDim.x + threadIdx.x, wi = w0 & 127;
+    const int64_t r_in = (wi & 3) * 32 + (wi >> 2);
+    const int64_t sa = stride >> 7, sa_r = sa / atoms_per_rowblock, sa_j = sa % atoms_per_rowblock;
+    int64_t rb = (w0 >> 7) / atoms_per_rowblock, j4 = (w0 >> 7) % atoms_per_rowblock;
+    float4 pnext = w0 < words ? __ldcs(jb.P + w0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t w = w0; w < words; w += stride) {
+        const float4 p = pnext;
+        if (w + stride < words) pnext = __ldcs(jb.P + w + stride);
+        const int64_t r = rb * 128 + r_in;                   // groups 4*j4 .. 4*j4+3 of view row r
         const uint4 u = philox_block(seed, jb.tid, (uint64_t)(r * atoms_per_rowblock + j4));
+        j4 += sa_j;
+        rb += sa_r;
+        if (j4 >= atoms_per_rowblock) {
+            j4 -= atoms_per_rowblock;
+            ++rb;
+        }
         const float pv[4] = {p.x, p.y, p.z, p.w};
         const uint32_t uv[4] = {u.x, u.y, u.z, u.w};
         uint32_t word = 0;
