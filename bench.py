@@ -1,14 +1,13 @@
 """Benchmark of the Quartet II NVFP4 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config mlp8b]
-                    [--schedule separate|fused|local] [--sweep] [--op fwd46_sq]
+                    [--schedule onepass|separate|fused|local] [--sweep] [--op fwd46_sq]
 
 A step is one pass of the whole hot path over one batch, for every linear layer of the
 workload: the forward quantizer on X and W (tensor max + RTN/4-6), the forward GEMM, MS-EDEN on
 dY (row and column views in one pass), on W (column view) and on X (column view) with their
-scale passes, and the dgrad and wgrad GEMMs -- the calls qt2_linear_fwd + qt2_linear_bwd make,
-issued here one C-ABI call at a time so that each kernel's duration is taken with CUDA events
-inside the timed region.
+scale passes, and the dgrad and wgrad GEMMs, issued one C-ABI call at a time so that each
+kernel's duration is taken with CUDA events inside the timed region.
 
 Workloads (nvfp4_quantized_b200.synth, seeded synthetic bf16 tensors):
   mlp8b (default)  the Llama-3-8B MLP at 16384 tokens: gate and up 4096 -> 14336 (one shared
@@ -20,10 +19,14 @@ Workloads (nvfp4_quantized_b200.synth, seeded synthetic bf16 tensors):
 Every step's inputs exceed L2 (126 MB) many times over, and two input sets alternate between
 steps, so no step starts with its inputs in L2.
 
-Schedules: separate (default: each linear as qt2_linear_fwd/bwd would run it); fused (NEXT-1:
-X's forward and MS-EDEN column views from one read, shared by linears that share X; W's two
-views made once before the timed steps, as for the micro-batches of one optimizer step); local
-(the forward with CTA-local scales, a different numeric contract).
+Schedules: onepass (default: every tensor of the step quantized once, both of its views from
+one read -- X's and W's forward and MS-EDEN column views through qt2_quant_fwd46_msedEN_col, X
+once for linears that read the same X, dY's two MS-EDEN views in one pass -- with a new seed
+every step, so the step does all of its work); separate (each linear as qt2_linear_fwd/bwd
+would run it: one quantizer call per view, X quantized per linear); fused (NEXT-1 with W's two
+views made once before the timed steps and one seed, as for the micro-batches of one optimizer
+step); local (the forward with CTA-local scales, a different numeric contract).  All but local
+produce the same bits for the same seed.
 
 Beside our numbers the line carries: torch bf16 matmuls on the same shapes and GPU (the pages'
 speed claims are relative to BF16), `e2e` through qt2_linear_fwd/bwd with every step's
@@ -176,6 +179,20 @@ def rank_input_seed(rank: int, set_index: int) -> int:
 
 
 # ---------------------------------------------------------------------------------------- step
+SCHEDULE_NOTE = {
+    "onepass": "per step and linear: X's forward (RTN+4/6) and MS-EDEN column views from one read "
+               "(once for linears that read the same X: gate and up), W's two views from one read, the "
+               "forward GEMM, MS-EDEN of dY (both views, one read), dgrad and wgrad GEMMs; a new seed every "
+               "step",
+    "separate": "per step and linear: fwd46(X), fwd46(W), forward GEMM, MS-EDEN of dY (both views), of W "
+                "(column view) and of X (column view), dgrad and wgrad GEMMs; a new seed every step",
+    "fused": "per step and linear: X's two views from one read (once per shared X), forward GEMM, MS-EDEN of "
+             "dY, dgrad and wgrad GEMMs; W's views made once before the timed steps and one seed for all "
+             "steps (the micro-batches of one optimizer step)",
+    "local": "as separate, with the forward's CTA-local scales (qt2_quant_fwd46_local, qt2_gemm_nvfp4_local)",
+}
+
+
 def step_flops(config: str) -> float:
     from nvfp4_quantized_b200 import synth
     return sum(3 * 2.0 * M * N * K for _, M, K, N, *_ in synth.stack_linears(config))
@@ -189,6 +206,9 @@ def call_names(linears, schedule: str):
         if schedule == "fused":
             calls = ([] if shared in seen_x else ["fused_x_views"]) + ["gemm_fwd", "msed_dy_both", "gemm_dgrad",
                                                                       "gemm_wgrad"]
+        elif schedule == "onepass":
+            calls = ([] if shared in seen_x else ["fused_x_views"]) + ["fused_w_views", "gemm_fwd", "msed_dy_both",
+                                                                      "gemm_dgrad", "gemm_wgrad"]
         elif schedule == "local":
             calls = ["fwd46_local_x", "fwd46_local_w", "gemm_fwd", "msed_dy_both", "msed_w_col", "msed_x_col",
                      "gemm_dgrad", "gemm_wgrad"]
@@ -207,7 +227,8 @@ def call_work(call: str, M: int, K: int, N: int):
     return "quant", {"fwd46_x": M * K * BYTES_FWD46, "fwd46_w": N * K * BYTES_FWD46,
                      "fwd46_local_x": M * K * BYTES_FWD46, "fwd46_local_w": N * K * BYTES_FWD46,
                      "msed_dy_both": M * N * BYTES_MSED_BOTH, "msed_w_col": N * K * BYTES_MSED_ONE,
-                     "msed_x_col": M * K * BYTES_MSED_ONE, "fused_x_views": M * K * BYTES_FUSED_X}[call]
+                     "msed_x_col": M * K * BYTES_MSED_ONE, "fused_x_views": M * K * BYTES_FUSED_X,
+                     "fused_w_views": N * K * BYTES_FUSED_X}[call]
 
 
 class LayerState:
@@ -229,6 +250,7 @@ class LayerState:
         self.ws_w = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(N, K, COL), dev)
         self.ws_x = Q.alloc_workspace(Q.qt2_quant_msedEN_workspace_size(M, K, COL), dev)
         self.ws_xv = Q.alloc_workspace(Q.qt2_quant_fwd46_msedEN_col_workspace_size(M, K), dev)
+        self.ws_wv = Q.alloc_workspace(Q.qt2_quant_fwd46_msedEN_col_workspace_size(N, K), dev)
         if local:
             self.vxl, self.vwl = Q.alloc_view_local(M, K, dev), Q.alloc_view_local(N, K, dev)
 
@@ -254,11 +276,16 @@ def make_step(Q, linears, sets, states, schedule, stream):
         for name, M, K, N, xk, dk, shared in linears:
             x, w, dy = sets[i % 2][name]
             st = states[name]
-            if schedule == "fused":
+            if schedule in ("fused", "onepass"):
                 if shared is None:
                     mark(j); j += 1
                     Q.qt2_quant_fwd46_msedEN_col(x, M, K, K, seed, Q.QT2_TID_X_COL, st.vx, st.v_x_col, st.ws_xv,
                                                  st.ws_xv.numel(), stream)
+                if schedule == "onepass":
+                    # W's forward view and MS-EDEN column view from one read, every step
+                    mark(j); j += 1
+                    Q.qt2_quant_fwd46_msedEN_col(w, N, K, K, seed, Q.QT2_TID_W_COL, st.vw, st.v_w_col, st.ws_wv,
+                                                 st.ws_wv.numel(), stream)
                 vx, vxc = (states[shared].vx, states[shared].v_x_col) if shared else (st.vx, st.v_x_col)
                 mark(j); j += 1
                 Q.qt2_gemm_nvfp4(vx, st.vw, M, N, K, 1.0, st.y, Q.QT2_DTYPE_BF16, N, stream)
@@ -413,8 +440,22 @@ def run_e2e(args, Q, linears, sets, dev, world, barrier):
                                  dy=torch.empty_like(dy), y=torch.empty((M, N), dtype=torch.bfloat16, device=dev),
                                  dx=torch.empty((M, K), dtype=torch.bfloat16, device=dev),
                                  dw=torch.empty((N, K), dtype=torch.float32, device=dev))
-    wsf = {n: Q.alloc_workspace(Q.qt2_linear_fwd_workspace_size(M, K, N), dev) for n, M, K, N, *_ in linears}
-    wsb = {n: Q.alloc_workspace(Q.qt2_linear_bwd_workspace_size(M, K, N), dev) for n, M, K, N, *_ in linears}
+    onepass = args.schedule == "onepass"
+    if onepass:
+        # the public calls of the one-pass schedule: both views of X (once per shared X) and of
+        # W from one read each, the forward GEMM, and the backward from those column views
+        views = {n: dict(vx=Q.alloc_view(M, K, dev), vxc=Q.alloc_view(K, M, dev), vw=Q.alloc_view(N, K, dev),
+                         vwc=Q.alloc_view(K, N, dev),
+                         wsx=Q.alloc_workspace(Q.qt2_quant_fwd46_msedEN_col_workspace_size(M, K), dev),
+                         wsw=Q.alloc_workspace(Q.qt2_quant_fwd46_msedEN_col_workspace_size(N, K), dev),
+                         wsb=Q.alloc_workspace(Q.qt2_linear_bwd_views_workspace_size(M, K, N), dev))
+                 for n, M, K, N, *_ in linears}
+        api = ("qt2_quant_fwd46_msedEN_col on X (once per shared X) and on W, qt2_gemm_nvfp4, "
+               "qt2_linear_bwd_views per linear")
+    else:
+        wsf = {n: Q.alloc_workspace(Q.qt2_linear_fwd_workspace_size(M, K, N), dev) for n, M, K, N, *_ in linears}
+        wsb = {n: Q.alloc_workspace(Q.qt2_linear_bwd_workspace_size(M, K, N), dev) for n, M, K, N, *_ in linears}
+        api = "qt2_linear_fwd + qt2_linear_bwd per linear"
     s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_cmp = [torch.cuda.Event() for _ in range(2)]
@@ -422,6 +463,20 @@ def run_e2e(args, Q, linears, sets, dev, world, barrier):
     used = [False, False]
 
     def compute(B, i, cs):
+        if onepass:
+            seed = 0xE2E0 + i
+            for name, M, K, N, xk, dk, shared in linears:
+                d, v = B[name], views[name]
+                vs = views[shared] if shared else v
+                if shared is None:
+                    Q.qt2_quant_fwd46_msedEN_col(d["x"], M, K, K, seed, Q.QT2_TID_X_COL, v["vx"], v["vxc"], v["wsx"],
+                                                 v["wsx"].numel(), cs)
+                Q.qt2_quant_fwd46_msedEN_col(d["w"], N, K, K, seed, Q.QT2_TID_W_COL, v["vw"], v["vwc"], v["wsw"],
+                                             v["wsw"].numel(), cs)
+                Q.qt2_gemm_nvfp4(vs["vx"], v["vw"], M, N, K, 1.0, d["y"], Q.QT2_DTYPE_BF16, N, cs)
+                Q.qt2_linear_bwd_views(d["dy"], M, K, N, seed, vs["vxc"], v["vwc"], d["dx"], d["dw"],
+                                       Q.QT2_DTYPE_F32, v["wsb"], v["wsb"].numel(), cs)
+            return
         for name, M, K, N, *_ in linears:
             d = B[name]
             Q.qt2_linear_fwd(d["x"], d["w"], M, K, N, d["y"], wsf[name], wsf[name].numel(), cs)
@@ -472,7 +527,7 @@ def run_e2e(args, Q, linears, sets, dev, world, barrier):
     e2e = {"value": job_tflops(world, flops, n, te), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": te / n,
            "pipeline": "3 streams (upload, compute, download), 2 device buffer sets; W resident",
-           "api": "qt2_linear_fwd + qt2_linear_bwd per linear"}
+           "api": api}
 
     # the same API calls on resident tensors
     cs = torch.cuda.current_stream(dev)
@@ -488,7 +543,7 @@ def run_e2e(args, Q, linears, sets, dev, world, barrier):
     torch.cuda.synchronize()
     tr = max_over_ranks(r_s.elapsed_time(r_e), world, dev)
     res = {"value": job_tflops(world, flops, n, tr), "unit": UNIT, "steps": n, "ms_per_step": tr / n,
-           "api": "qt2_linear_fwd + qt2_linear_bwd per linear, inputs and outputs resident"}
+           "api": api + ", inputs and outputs resident"}
     assert Q.qt2_device_status() == 0
     return e2e, res
 
@@ -644,8 +699,11 @@ def main():
     ap.add_argument("--cpu-w-rows", type=int, default=4096)
     ap.add_argument("--cpu-tokens-1t", type=int, default=128)
     ap.add_argument("--cpu-w-rows-1t", type=int, default=1024)
-    ap.add_argument("--schedule", choices=["separate", "fused", "local"], default="separate",
-                    help="fused: X's forward and column views from one read (qt2_quant_fwd46_msedEN_col) and "
+    ap.add_argument("--schedule", choices=["onepass", "separate", "fused", "local"], default="onepass",
+                    help="onepass (default): every tensor quantized once a step, both of its views from one read "
+                         "(qt2_quant_fwd46_msedEN_col on X and on W; MS-EDEN of dY, both views); separate: each "
+                         "linear as qt2_linear_fwd/bwd runs it (one quantizer call per view, X per linear); "
+                         "fused: X's forward and column views from one read (qt2_quant_fwd46_msedEN_col) and "
                          "W's forward and column views made once and reused by every step, as micro-batches of "
                          "one optimizer step; local: the forward with CTA-local scales (qt2_quant_fwd46_local, "
                          "qt2_gemm_nvfp4_local), a different numeric contract")
@@ -728,7 +786,8 @@ def main():
                    "flop_per_step": flops,
                    "parallelism": f"dp{world}: every rank its own token batch, no collective on the path",
                    "l2": "inputs larger than L2: every step reads several GB, two input sets alternate",
-                   "output": "Y bf16, dX bf16, dW fp32", "schedule": args.schedule},
+                   "output": "Y bf16, dX bf16, dW fp32", "schedule": args.schedule,
+                   "schedule_calls": SCHEDULE_NOTE[args.schedule]},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp4_peak, "traffic": traffic,
                      "kernel": f"gemm_nvfp4_pair_kernel (all {n_gemm} GEMM launches of the step: their FLOPs over "

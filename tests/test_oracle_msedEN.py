@@ -271,3 +271,85 @@ def test_flushed_and_zero_views():
     tiny = _bf16(np.full((4, 128), 1e-33, np.float32))
     t = O.msedEN(tiny, 0, 1, "row")
     assert np.all(t.amax_g < 2.0 ** -100) and np.all(t.scales == 0) and t.g == 1.0
+
+
+def test_scale_sr_outcomes_enumerated_on_one_128_block():
+    """Brute force over every outcome of the stochastic scale rounding of one 128-element block
+    (the digest's "Method": FP8 group scales rounded stochastically; the EDEN factor folded into
+    them).  Row 0 of a 2 x 128 tensor has 8 groups whose scale t = S p / g lies in the E4M3
+    normal range, each rounded down or up; row 1 is 2e-5 times smaller, so its scales fall below
+    2^-6 and take RNE (one outcome).  Enumerating the 2^8 joint outcomes with their
+    probabilities gives the exact expectation of the dequantized block; it must carry the EDEN
+    identity <E[xhat], y> = <y, y>.  Then the oracle's draws over 8192 SR keys (tensor ids; the
+    seed, hence the rotation, fixed) must land only on enumerated outcomes, with the enumerated
+    frequencies (per group, per pair of groups, and a chi-square over the 256 joint outcomes),
+    and their mean must match the enumerated expectation."""
+    from scipy.stats import chi2, norm
+    rng = np.random.default_rng(21)
+    xf = rng.standard_normal((2, 128)).astype(np.float32)
+    xf[1] *= 2e-5
+    x = _bf16(xf)
+    seed = 77
+    y = _rotated(x, seed).astype(np.float64)
+    e4 = np.array([O.e4m3_value(c) for c in range(127)])
+    ref = O.msedEN(x, seed, 1, "row")
+    g = np.float32(ref.g)
+    ginv = np.float32(np.float32(1.0) / g)
+    val = np.array([O.e2m1_value(c) for c in range(16)])[_unpack(ref.codes)]   # codes do not depend on the key
+    t = (ref.P * ginv).astype(np.float32).astype(np.float64)                   # [2][8]
+    assert np.all(t[0] >= 2.0 ** -6) and np.all(t[1] < 2.0 ** -6)
+    lo = np.array([e4[e4 <= v].max() for v in t[0]])
+    hi = np.array([e4[e4 >= v].min() for v in t[0]])
+    assert np.all(hi > lo)
+    p_hi = (t[0] - lo) / (hi - lo)
+    rne1 = np.array([O.e4m3_value(O.e4m3_rne(float(v))) for v in t[1]])
+
+    # exact expectation by enumeration of the 256 joint outcomes
+    combos = (np.arange(256)[:, None] >> np.arange(8)[None, :]) & 1          # [256][8], 1 = rounded up
+    prob = np.prod(np.where(combos == 1, p_hi, 1 - p_hi), axis=1)
+    assert abs(prob.sum() - 1.0) < 1e-12
+    scale0 = np.where(combos == 1, hi, lo)                                    # [256][8]
+    xhat0 = val[0][None, :] * np.repeat(scale0, 16, axis=1) * float(g)        # [256][128]
+    E0 = prob @ xhat0
+    # closed form of the same expectation: the SR of each scale is unbiased
+    assert np.allclose(E0, val[0] * np.repeat(t[0], 16) * float(g), rtol=1e-12, atol=0)
+    # the EDEN identity on the expectation (S folded into the scales): <E[xhat], y> = <y, y>
+    yy = float(y[0] @ y[0])
+    assert abs(float(E0 @ y[0]) - yy) <= 1e-5 * yy
+
+    # the oracle's draws over 8192 keys
+    B = 8192
+    counts = np.zeros(256, np.int64)
+    s1 = np.zeros(128)
+    for tid in range(B):
+        v = O.msedEN(x, seed, 1000 + tid, "row")
+        assert np.array_equal(v.codes, ref.codes) and v.g == g
+        s = np.array([O.e4m3_value(c) for c in v.scales.ravel()]).reshape(2, 8)
+        assert np.array_equal(s[1], rne1)
+        up = s[0] == hi
+        assert np.all(up | (s[0] == lo))
+        counts[int(np.sum(up.astype(np.int64) << np.arange(8)))] += 1
+        s1 += val[0] * np.repeat(s[0], 16) * float(g)
+    thr = norm.isf(0.001 / (2 * (8 + 28 + 128)))      # Bonferroni over every z below
+    n_up = (combos * counts[:, None]).sum(axis=0)
+    z1 = (n_up - B * p_hi) / np.sqrt(B * p_hi * (1 - p_hi))
+    assert np.max(np.abs(z1)) < thr, z1
+    for a in range(8):
+        for b in range(a + 1, 8):
+            pj = p_hi[a] * p_hi[b]
+            nj = counts[(combos[:, a] == 1) & (combos[:, b] == 1)].sum()
+            assert abs(nj - B * pj) / np.sqrt(B * pj * (1 - pj)) < thr, (a, b)
+    exp_c = B * prob
+    keep = exp_c >= 5
+    stat = np.sum((counts[keep] - exp_c[keep]) ** 2 / exp_c[keep])
+    rest_o, rest_e = counts[~keep].sum(), exp_c[~keep].sum()
+    dof = int(keep.sum()) - 1
+    if rest_e > 0:
+        stat += (rest_o - rest_e) ** 2 / rest_e
+        dof += 1
+    assert chi2.sf(stat, dof) > 1e-4, (stat, dof)
+    # mean of the draws against the enumerated expectation, per coordinate
+    var = prob @ (xhat0 - E0) ** 2
+    nz = var > 0
+    zc = (s1 / B - E0)[nz] / np.sqrt(var[nz] / B)
+    assert np.max(np.abs(zc)) < thr
