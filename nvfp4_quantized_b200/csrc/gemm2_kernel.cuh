@@ -159,7 +159,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const float *__restrict__ gA, const float *__restrict__ gB, float alpha,
-                           void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype, int local) {
+                           void *__restrict__ Cout, int64_t ldc, int M, int N, int K, int c_dtype, int local,
+                           int m_fast) {
     using Cfg = Gemm2Cfg;
     constexpr int S = Cfg::kStages;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -171,7 +172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_pn = N >> 8, tiles = (M >> 8) * num_pn;
+    const int num_pm = M >> 8, num_pn = N >> 8, tiles = num_pm * num_pn;
     const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
     const int nkb = K >> 6, nks = (nkb + 3) >> 2;
     const int my_tiles = tiles > cluster_id ? (tiles - 1 - cluster_id) / num_clusters + 1 : 0;
@@ -201,11 +202,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // Tile order.  The ~74 tiles in flight at a time read their A row blocks and B row blocks
+    // from L2; the operand whose row blocks they share should be the one that is re-read.  With
+    // m_fast the tile index runs over M first, so the tiles in flight cover all of a small A and a
+    // few B row blocks, and B streams from DRAM once (instead of once per row of tiles when A is
+    // the smaller operand and N is wide).
+    auto tile_coords = [&](int tile, int &pm, int &pn) {
+        if (m_fast) {
+            pn = tile / num_pm;
+            pm = tile - pn * num_pm;
+        } else {
+            pm = tile / num_pn;
+            pn = tile - pm * num_pn;
+        }
+    };
     auto stage_tile = [&](int it, int &pm, int &pn, int &ks) {
         const int tile = cluster_id + (it / nks) * num_clusters;
         ks = it % nks;
-        pm = tile / num_pn;
-        pn = tile - pm * num_pn;
+        tile_coords(tile, pm, pn);
     };
 
     int issued = 0;     // producer: stages whose loads were issued
@@ -315,7 +329,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             if (!mbar_wait_warp(acc_full, t_iter & 1)) break;
             tc_fence_after();
             const int tile = cluster_id + t_iter * num_clusters;
-            const int pm = tile / num_pn, pn = tile - pm * num_pn;
+            int pm, pn;
+            tile_coords(tile, pm, pn);
             const int64_t row = (int64_t)pm * 256 + rank * 128 + quad * 32 + lane;
             const int64_t col = (int64_t)pn * 256 + cb;
             // tensor scales: one each, or (CTA-local views) one per 128 rows of A and of B

@@ -288,9 +288,11 @@ cudaError_t launch_gemm_nvfp4_pair(const CUtensorMap &tmA, const CUtensorMap &tm
     if (attr_err != cudaSuccess) return attr_err;
     const int64_t tiles = (M / 256) * (N / 256);
     const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(tiles, sm_count() / 2));
+    // run the tiles along M first when A is the smaller operand (see the kernel's tile order)
+    const int m_fast = M < N ? 1 : 0;
     gemm_nvfp4_pair_kernel<<<(unsigned)(2 * clusters), Gemm2Cfg::kThreads, Gemm2Cfg::kSmemBytes, s>>>(
         tmA, tmB, tmSFA, tmSFB, a.tensor_scale, b.tensor_scale, alpha, c, ldc, (int)M, (int)N, (int)K, c_dtype,
-        local);
+        local, m_fast);
     return cudaGetLastError();
 }
 

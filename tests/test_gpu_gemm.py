@@ -52,8 +52,9 @@ def _x(R, C, seed, scale=1.0):
 SHAPES = [(128, 128, 128), (128, 256, 256), (256, 256, 256), (384, 640, 1152), (256, 512, 2048), (128, 384, 4224),
           (256, 256, 8192),
           # M and N multiples of 256 run on SM pairs: several tiles each way, a K tail (4224 = 16.5 x 256),
-          # and more tiles (16 x 16) than resident pairs, so each pair loops over tiles
-          (512, 768, 1024), (768, 512, 4224), (4096, 4096, 512)]
+          # and more tiles (16 x 16) than resident pairs, so each pair loops over tiles; M < N with
+          # more tiles than pairs (the tile order that runs along M first)
+          (512, 768, 1024), (768, 512, 4224), (4096, 4096, 512), (1024, 9728, 768)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
