@@ -65,7 +65,9 @@ typedef enum {
     QT2_ERR_CUDA = -5,        /* a CUDA runtime/driver call or launch failed */
     QT2_ERR_TIMEOUT = -6,     /* a device-side bounded wait gave up (see qt2_device_status) */
     QT2_ERR_DEVICE = -7,      /* no device, or the current device is not sm_100 */
-    QT2_ERR_NONFINITE = -8    /* device-side: an input held inf or NaN (see qt2_device_status) */
+    QT2_ERR_NONFINITE = -8,   /* device-side: an input held inf or NaN (see qt2_device_status) */
+    QT2_ERR_BOUNDS = -9       /* device-side, checked build only: a store index left its output
+                                 array; the store was skipped (see qt2_build_checked) */
 } qt2_status;
 
 enum { QT2_LAYOUT_ROW = 1, QT2_LAYOUT_COL = 2, QT2_LAYOUT_BOTH = 3 };
@@ -85,7 +87,9 @@ QT2_API const char *qt2_status_string(qt2_status s);
 
 /* Reads and clears the library's device-side status word after synchronizing `stream`.
  * *code = 0 when no kernel reported a problem; QT2_ERR_TIMEOUT when a bounded wait gave up;
- * QT2_ERR_NONFINITE when a quantizer met inf or NaN in its input (the first report wins).
+ * QT2_ERR_NONFINITE when a quantizer met inf or NaN in its input; QT2_ERR_BOUNDS (checked build
+ * only) when a kernel skipped a store that would have left its output array (the first report
+ * wins).
  * Synchronizes the stream; meant for tests and debugging, not the hot path. */
 QT2_API qt2_status qt2_device_status(qt2_stream_t stream, int *code);
 
@@ -322,6 +326,22 @@ QT2_API qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream);
  * --------------------------------------------------------------------------------------- */
 QT2_API qt2_status qt2_selftest_division(uint32_t exp_lo, uint32_t exp_hi, unsigned long long *mismatches,
                                          qt2_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Checked build.  The same sources compiled with QT2_CHECKED give libqt2_checked.so (built beside
+ * libqt2.so, the same entry points): every global store of every kernel first checks that the
+ * bytes it writes lie inside the output array the call was given (the view's codes, scales or
+ * pre-scales, the GEMM's C rows) and, if not, skips the store and records QT2_ERR_BOUNDS in the
+ * device status word.  It runs slower and is meant for testing and debugging, not the hot path.
+ * qt2_build_checked returns 1 in the checked build, 0 in the product build.
+ * qt2_selftest_bounds enqueues one kernel that stores one byte through that check into a
+ * 64-byte array of the library's own, at offset 40 against a stated extent of 32 bytes: the
+ * checked build skips the store and records QT2_ERR_BOUNDS (read it with qt2_device_status);
+ * the product build, which has no checks, makes the store (still inside the array) and records
+ * nothing.  Enqueued on `stream`.
+ * --------------------------------------------------------------------------------------- */
+QT2_API int qt2_build_checked(void);
+QT2_API qt2_status qt2_selftest_bounds(qt2_stream_t stream);
 
 #ifdef __cplusplus
 }

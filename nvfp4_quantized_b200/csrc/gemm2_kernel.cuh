@@ -346,6 +346,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            // checked build: this thread's 128 outputs must lie inside C ((M - 1) * ldc + N elements)
+            const int64_t esz = c_dtype == QT2_DTYPE_F32 ? 4 : 2;
+            if (!QT2_STORE_OK(static_cast<uint8_t *>(Cout) + (row * ldc + col) * esz, 128 * esz, Cout,
+                              ((int64_t)(M - 1) * ldc + N) * esz))
+                continue;
             // 32-byte stores (each fills whole 32-byte sectors of its row) when C's rows are
             // 32-byte aligned, else 16-byte stores
             if (c_dtype == QT2_DTYPE_F32) {

@@ -155,6 +155,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (acc_ok) {
         const int64_t row = m0 + warp * 32 + lane;
         const uint32_t t_row = t_acc + ((uint32_t)(warp * 32) << 16);
+        // checked build: this thread's BN outputs must lie inside C ((M - 1) * ldc + N elements,
+        // M and N from the grid); the TMEM loads below stay warp-collective either way
+        const int64_t esz = c_dtype == QT2_DTYPE_F32 ? 4 : 2;
+        const bool st_ok = QT2_STORE_OK(static_cast<uint8_t *>(Cout) + (row * ldc + n0) * esz, BN * esz, Cout,
+                                        (((int64_t)gridDim.y * kGemmBM - 1) * ldc + (int64_t)gridDim.x * BN) * esz);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
             // tensor scales: one each, or (CTA-local views) one per 128 rows of A and of B
@@ -162,6 +167,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t v[16];
             tmem_ld_32x32b_x16(t_row + c, v);
             tmem_ld_wait();
+            if (!st_ok) continue;
             if (c_dtype == QT2_DTYPE_F32) {
                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(Cout) + row * ldc + n0 + c);
 #pragma unroll

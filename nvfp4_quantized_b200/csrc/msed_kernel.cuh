@@ -310,12 +310,20 @@ __device__ __forceinline__ void sr_vector(const uint64_t (&P)[32], float g, floa
 // Codes of the thread's groups {2h, 2h+1} and {4+2h, 5+2h} of a 128-block starting at group j0
 // of view row vr (codes_row points at the block's first code byte); pre-scales in tensor-core
 // scale order.
+// codes_base and n_elems (the view's element count) bound the stores in the checked build.
 __device__ __forceinline__ void msed_store(uint8_t *codes_row, float *P_base, int64_t vr, int64_t j0, int64_t VC,
-                                           int h, const uint32_t (&cw)[8], const float (&Pq)[4]) {
-    *reinterpret_cast<uint4 *>(codes_row + 16 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    *reinterpret_cast<uint4 *>(codes_row + 32 + 16 * h) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-    *reinterpret_cast<float2 *>(P_base + sf_offset(vr, j0 + 2 * h, VC)) = make_float2(Pq[0], Pq[1]);
-    *reinterpret_cast<float2 *>(P_base + sf_offset(vr, j0 + 4 + 2 * h, VC)) = make_float2(Pq[2], Pq[3]);
+                                           int h, const uint32_t (&cw)[8], const float (&Pq)[4],
+                                           const uint8_t *codes_base, int64_t n_elems) {
+    (void)codes_base;
+    (void)n_elems;
+    uint8_t *const c0 = codes_row + 16 * h, *const c1 = codes_row + 32 + 16 * h;
+    float *const p0 = P_base + sf_offset(vr, j0 + 2 * h, VC), *const p1 = P_base + sf_offset(vr, j0 + 4 + 2 * h, VC);
+    if (QT2_STORE_OK(c0, 16, codes_base, n_elems >> 1))
+        *reinterpret_cast<uint4 *>(c0) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    if (QT2_STORE_OK(c1, 16, codes_base, n_elems >> 1))
+        *reinterpret_cast<uint4 *>(c1) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    if (QT2_STORE_OK(p0, 8, P_base, (n_elems >> 4) * 4)) *reinterpret_cast<float2 *>(p0) = make_float2(Pq[0], Pq[1]);
+    if (QT2_STORE_OK(p1, 8, P_base, (n_elems >> 4) * 4)) *reinterpret_cast<float2 *>(p1) = make_float2(Pq[2], Pq[3]);
 }
 
 // What one launch of the rotation producer emits per view (row view: [R][C]; column view: the
@@ -475,9 +483,12 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
                 release(s, i);
                 const int64_t vr = r0 + u;
                 uint8_t *const vcodes = row_codes + vr * (C >> 1) + (c0 >> 1);
-                *reinterpret_cast<uint4 *>(vcodes + 32 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                *reinterpret_cast<uint4 *>(vcodes + 32 * h + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-                *reinterpret_cast<uint32_t *>(out.row_scales + sf_offset(vr, (c0 >> 4) + 4 * h, C)) = scw;
+                uint8_t *const sdst = out.row_scales + sf_offset(vr, (c0 >> 4) + 4 * h, C);
+                if (QT2_STORE_OK(vcodes + 32 * h, 32, row_codes, R * (C >> 1))) {
+                    *reinterpret_cast<uint4 *>(vcodes + 32 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    *reinterpret_cast<uint4 *>(vcodes + 32 * h + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                }
+                if (QT2_STORE_OK(sdst, 4, out.row_scales, R * (C >> 4))) *reinterpret_cast<uint32_t *>(sdst) = scw;
                 continue;
             }
         }
@@ -542,12 +553,12 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             uint32_t cw[8];
             float Pq[4];
             msed_vector(P, sg, nsg, nz, cw, Pq, amax);
-            msed_store(vcodes, rows ? row_P : col_P, vr, b0 >> 4, VC, h, cw, Pq);
+            msed_store(vcodes, rows ? row_P : col_P, vr, b0 >> 4, VC, h, cw, Pq, rows ? row_codes : col_codes, R * C);
         } else if constexpr (MODE == kModeFwdRowEdenCol) {   // column warps (rows returned above)
             uint32_t cw[8];
             float Pq[4];
             msed_vector(P, sg, nsg, nz, cw, Pq, amax);
-            msed_store(vcodes, col_P, vr, b0 >> 4, VC, h, cw, Pq);
+            msed_store(vcodes, col_P, vr, b0 >> 4, VC, h, cw, Pq, col_codes, R * C);
         } else if constexpr (MODE == kModeMax) {
             rotate_tail(P, sg, nsg);
 #pragma unroll
@@ -564,12 +575,15 @@ __global__ void __launch_bounds__(MsedCfg::kThreads, 1)
             uint32_t cw[8], scq[4];
             sr_vector(P, rows ? g_r : g_c, rows ? g6_r : g6_c, rows ? zero_r : zero_c, seed,
                       rows ? out.tid_row : out.tid_col, e_base, cw, scq, amax);
-            *reinterpret_cast<uint4 *>(vcodes + 16 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            *reinterpret_cast<uint4 *>(vcodes + 32 + 16 * h) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            const uint8_t *const cb = rows ? row_codes : col_codes;
+            if (QT2_STORE_OK(vcodes + 16 * h, 16, cb, (R * C) >> 1))
+                *reinterpret_cast<uint4 *>(vcodes + 16 * h) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            if (QT2_STORE_OK(vcodes + 32 + 16 * h, 16, cb, (R * C) >> 1))
+                *reinterpret_cast<uint4 *>(vcodes + 32 + 16 * h) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
             uint8_t *const sb = rows ? out.row_scales : out.col_scales;
-            *reinterpret_cast<uint16_t *>(sb + sf_offset(vr, (b0 >> 4) + 2 * h, VC)) = (uint16_t)(scq[0] | (scq[1] << 8));
-            *reinterpret_cast<uint16_t *>(sb + sf_offset(vr, (b0 >> 4) + 4 + 2 * h, VC)) =
-                (uint16_t)(scq[2] | (scq[3] << 8));
+            uint8_t *const s0 = sb + sf_offset(vr, (b0 >> 4) + 2 * h, VC), *const s1 = sb + sf_offset(vr, (b0 >> 4) + 4 + 2 * h, VC);
+            if (QT2_STORE_OK(s0, 2, sb, (R * C) >> 4)) *reinterpret_cast<uint16_t *>(s0) = (uint16_t)(scq[0] | (scq[1] << 8));
+            if (QT2_STORE_OK(s1, 2, sb, (R * C) >> 4)) *reinterpret_cast<uint16_t *>(s1) = (uint16_t)(scq[2] | (scq[3] << 8));
         }
     }
     if constexpr (MODE != kModeSr) {

@@ -22,6 +22,26 @@ __device__ int g_device_status = 0;
 
 __device__ __forceinline__ void set_device_error(int code) { atomicCAS(&g_device_status, 0, code); }
 
+// ------------------------------------------------------------------------------------------
+// Store checks of the checked build (compiled with -DQT2_CHECKED into libqt2_checked.so): every
+// global store of the kernels' outputs first checks that its bytes [p, p + bytes) lie inside the
+// output array [base, base + extent) the launch was given; a store that would leave it is
+// skipped and QT2_ERR_BOUNDS recorded in the status word.  In the product build the check is
+// the constant true and costs nothing.
+// ------------------------------------------------------------------------------------------
+#ifdef QT2_CHECKED
+__device__ __noinline__ bool store_in_bounds(const void *p, uint64_t bytes, const void *base, uint64_t extent) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+    if (a >= b && a - b <= extent && bytes <= extent - (a - b)) return true;
+    set_device_error(QT2_ERR_BOUNDS);
+    return false;
+}
+#define QT2_STORE_OK(p, bytes, base, extent) \
+    (::qt2::store_in_bounds((p), (uint64_t)(bytes), (base), (uint64_t)(extent)))
+#else
+#define QT2_STORE_OK(p, bytes, base, extent) true
+#endif
+
 // Upper bound of any single wait inside a kernel (ns).  A correct launch never comes close.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 

@@ -139,6 +139,15 @@ __global__ void selftest_wait_kernel() {
     if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0);
 }
 
+// Self-test of the checked build's store check: one byte at offset 40 of a 64-byte array,
+// checked against a stated extent of 32 bytes (skipped and reported in the checked build; made,
+// inside the array, in the product build, which has no checks).
+__device__ unsigned char g_bounds_probe[64];
+__global__ void selftest_bounds_kernel() {
+    unsigned char *const p = g_bounds_probe + 40;
+    if (threadIdx.x == 0 && QT2_STORE_OK(p, 1, g_bounds_probe, 32)) *p = 1;
+}
+
 // Self-test of the quantizers' division shortcuts: for every binary32 value x whose biased
 // exponent lies in [e_lo, e_hi] (every significand), rcp_rn(x) against the IEEE reciprocal
 // (counted in mismatches[0]) and div6_rn(x) against the IEEE quotient x/6 (mismatches[1]).
@@ -650,6 +659,7 @@ const char *qt2_status_string(qt2_status s) {
         case QT2_ERR_TIMEOUT: return "device-side wait timed out";
         case QT2_ERR_DEVICE: return "no sm_100 device";
         case QT2_ERR_NONFINITE: return "input holds inf or NaN";
+        case QT2_ERR_BOUNDS: return "a kernel store left its output array (checked build; store skipped)";
     }
     return "unknown status";
 }
@@ -846,6 +856,25 @@ qt2_status qt2_selftest_wait_timeout(qt2_stream_t stream) {
     if (fa == kFaultFail) return QT2_ERR_CUDA;
     if (fa == kFaultSkip) return QT2_OK;
     selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return from_cuda(cudaGetLastError());
+}
+
+int qt2_build_checked(void) {
+#ifdef QT2_CHECKED
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+qt2_status qt2_selftest_bounds(qt2_stream_t stream) {
+    QT2_TRACE();
+    qt2_status st = check_device();
+    if (st != QT2_OK) return st;
+    const int fa = fault_at("launch");
+    if (fa == kFaultFail) return QT2_ERR_CUDA;
+    if (fa == kFaultSkip) return QT2_OK;
+    selftest_bounds_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
     return from_cuda(cudaGetLastError());
 }
 

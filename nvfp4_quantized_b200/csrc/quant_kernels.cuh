@@ -387,12 +387,14 @@ __global__ void __launch_bounds__(256) fwd46_coop_kernel(const uint16_t *__restr
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t code0, code1;
         const uint32_t sc = fwd46_group(w, kc, tab_d, tab_r, code0, code1);
-        *reinterpret_cast<uint2 *>(codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8) = make_uint2(code0, code1);
+        uint8_t *const cdst = codes + r * (uint64_t)(C >> 1) + (uint64_t)q * 8;
+        if (QT2_STORE_OK(cdst, 8, codes, R * (C >> 1))) *reinterpret_cast<uint2 *>(cdst) = make_uint2(code0, code1);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-        if ((lane & 3) == 0)
-            *reinterpret_cast<uint32_t *>(scales + sf_offset((int64_t)r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        uint8_t *const sdst = scales + sf_offset((int64_t)r, q, C);
+        if ((lane & 3) == 0 && QT2_STORE_OK(sdst, 4, scales, R * (C >> 4)))
+            *reinterpret_cast<uint32_t *>(sdst) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
         gi = gn;
         r = rn;
         q = qn;
@@ -459,7 +461,7 @@ __global__ void __cluster_dims__(kLocalCluster, 1, 1) __launch_bounds__(kLocalTh
     const float A = __uint_as_float(bmax);
     const float g = (A >= kTiny) ? __fdiv_rn(A, kFwd46Denominator) : 1.0f;
     Fwd46Consts kc = fwd46_consts(g);
-    if (rank == 0 && threadIdx.x == 0) g_blocks[blk] = g;
+    if (rank == 0 && threadIdx.x == 0 && QT2_STORE_OK(g_blocks + blk, 4, g_blocks, (R >> 7) * 4)) g_blocks[blk] = g;
     __shared__ float tab_d[128], tab_r[129];
     fwd46_tables(g, tab_d, tab_r);
     __syncthreads();
@@ -476,12 +478,14 @@ __global__ void __cluster_dims__(kLocalCluster, 1, 1) __launch_bounds__(kLocalTh
         const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint32_t code0, code1;
         const uint32_t sc = fwd46_group(w, kc, tab_d, tab_r, code0, code1);
-        *reinterpret_cast<uint2 *>(codes + r * (C >> 1) + (int64_t)q * 8) = make_uint2(code0, code1);
+        uint8_t *const cdst = codes + r * (C >> 1) + (int64_t)q * 8;
+        if (QT2_STORE_OK(cdst, 8, codes, R * (C >> 1))) *reinterpret_cast<uint2 *>(cdst) = make_uint2(code0, code1);
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-        if ((lane & 3) == 0)
-            *reinterpret_cast<uint32_t *>(scales + sf_offset(r, q, C)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        uint8_t *const sdst = scales + sf_offset(r, q, C);
+        if ((lane & 3) == 0 && QT2_STORE_OK(sdst, 4, scales, R * (C >> 4)))
+            *reinterpret_cast<uint32_t *>(sdst) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
         rr += step_r;
         q += step_q;
         if (q >= G) {
@@ -558,8 +562,9 @@ __global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restric
         const uint32_t code0 = pick4 ? c4[0] : c6[0], code1 = pick4 ? c4[1] : c6[1];
         const uint32_t sc = pick4 ? s4.code : s6.code;
         // row view: row r, group q
-        *reinterpret_cast<uint2 *>(row_codes + r * (C >> 1) + q * 8) = make_uint2(code0, code1);
-        row_scales[sf_offset(r, q, C)] = (uint8_t)sc;
+        uint8_t *const rc = row_codes + r * (C >> 1) + q * 8, *const rs = row_scales + sf_offset(r, q, C);
+        if (QT2_STORE_OK(rc, 8, row_codes, R * (C >> 1))) *reinterpret_cast<uint2 *>(rc) = make_uint2(code0, code1);
+        if (QT2_STORE_OK(rs, 1, row_scales, R * (C >> 4))) *rs = (uint8_t)sc;
         // column view: row 16q + j of the transpose, group rb; nibble i = element (16rb + i, 16q + j)
         const uint64_t mine = ((uint64_t)code1 << 32) | code0;
         uint64_t tr = 0;
@@ -569,8 +574,10 @@ __global__ void __launch_bounds__(256) fwd46_sq_kernel(const uint16_t *__restric
             tr |= ((other >> (4 * j)) & 0xFull) << (4 * i);
         }
         const int64_t cr = q * 16 + j;
-        *reinterpret_cast<uint2 *>(col_codes + cr * (R >> 1) + rb * 8) = make_uint2((uint32_t)tr, (uint32_t)(tr >> 32));
-        col_scales[sf_offset(cr, rb, R)] = (uint8_t)sc;
+        uint8_t *const cc = col_codes + cr * (R >> 1) + rb * 8, *const cs = col_scales + sf_offset(cr, rb, R);
+        if (QT2_STORE_OK(cc, 8, col_codes, C * (R >> 1)))
+            *reinterpret_cast<uint2 *>(cc) = make_uint2((uint32_t)tr, (uint32_t)(tr >> 32));
+        if (QT2_STORE_OK(cs, 1, col_scales, C * (R >> 4))) *cs = (uint8_t)sc;
     }
 }
 
@@ -638,7 +645,7 @@ __global__ void __launch_bounds__(256) msed_finalize_kernel(FinalizeJob j0, Fina
             const uint32_t s = (v < kSrCutoff) ? e4m3_rne(v) : e4m3_sr(v, uv[k]);
             word |= s << (8 * k);
         }
-        jb.scale_words[w] = word;
+        if (QT2_STORE_OK(jb.scale_words + w, 4, jb.scale_words, words * 4)) jb.scale_words[w] = word;
     }
 }
 

@@ -16,12 +16,14 @@ from dataclasses import dataclass
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libqt2.so")
+# QT2_LIBRARY=checked loads the checked build (every kernel store checked against its output
+# array, include/qt2.h); anything else, or unset, the product library
+LIB_PATH = os.path.join(_PKG, "libqt2_checked.so" if os.environ.get("QT2_LIBRARY") == "checked" else "libqt2.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "qt2.h")
 
 QT2_OK = 0
 QT2_ERR_INVALID_ARG, QT2_ERR_SHAPE, QT2_ERR_ALIGN, QT2_ERR_WORKSPACE = -1, -2, -3, -4
-QT2_ERR_CUDA, QT2_ERR_TIMEOUT, QT2_ERR_DEVICE, QT2_ERR_NONFINITE = -5, -6, -7, -8
+QT2_ERR_CUDA, QT2_ERR_TIMEOUT, QT2_ERR_DEVICE, QT2_ERR_NONFINITE, QT2_ERR_BOUNDS = -5, -6, -7, -8, -9
 QT2_LAYOUT_ROW, QT2_LAYOUT_COL, QT2_LAYOUT_BOTH = 1, 2, 3
 QT2_DTYPE_BF16, QT2_DTYPE_F32 = 0, 1
 QT2_TID_SIGNS, QT2_TID_DY_ROW, QT2_TID_DY_COL, QT2_TID_W_COL, QT2_TID_X_COL = 0, 1, 2, 3, 4
@@ -79,6 +81,8 @@ def lib() -> ctypes.CDLL:
                 "qt2_selftest_wait_timeout": (i32, [vp]),
                 "qt2_set_fault_hook": (None, [FaultHookC, vp]),
                 "qt2_selftest_division": (i32, [u32, u32, vp, vp]),
+                "qt2_build_checked": (i32, []),
+                "qt2_selftest_bounds": (i32, [vp]),
                 "qt2_gemm_nvfp4_local": (i32, [pv, pv, i64, i64, i64, f32, vp, i32, i64, vp]),
                 "qt2_quant_fwd46_sq_workspace_size": (i32, [i64, i64, psz]),
                 "qt2_quant_fwd46_sq": (i32, [vp, i64, i64, i64, pv, pv, vp, sz, vp]),
@@ -360,6 +364,16 @@ def qt2_selftest_division(exp_lo: int, exp_hi: int, stream=None) -> tuple[int, i
     _check("qt2_selftest_division", lib().qt2_selftest_division(exp_lo, exp_hi, cnt.data_ptr(), _stream(stream)))
     r, d = cnt.tolist()
     return int(r), int(d)
+
+
+def qt2_build_checked() -> bool:
+    """True when the loaded library is the checked build (QT2_LIBRARY=checked)."""
+    return bool(lib().qt2_build_checked())
+
+
+def qt2_selftest_bounds(stream=None) -> None:
+    """Enqueue the store-check self-test (the checked build records QT2_ERR_BOUNDS)."""
+    _check("qt2_selftest_bounds", lib().qt2_selftest_bounds(_stream(stream)))
 
 
 def qt2_selftest_wait_timeout(stream=None) -> None:

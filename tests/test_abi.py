@@ -21,7 +21,7 @@ def L():
 
 def test_exports_every_header_function(L):
     names = qt2.header_functions()
-    assert len(names) == 26
+    assert len(names) == 28
     out = subprocess.run(["nm", "-D", "--defined-only", qt2.LIB_PATH], capture_output=True, text=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     missing = [n for n in names if n not in exported]
@@ -32,6 +32,20 @@ def test_exports_every_header_function(L):
     assert {e for e in exported if e.startswith("qt2")} == set(names)
 
 
+def test_checked_build_exports_the_same_abi(L):
+    """libqt2_checked.so (QT2_CHECKED: every kernel store checked) has exactly the product
+    library's entry points and says which build it is; the product library says it is not."""
+    path = qbuild.build(checked=True)
+    names = qt2.header_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert {e for e in exported if e.startswith("qt2")} == set(names)
+    C = ctypes.CDLL(path)
+    assert C.qt2_build_checked() == 1
+    assert L.qt2_build_checked() == 0
+    assert qt2.qt2_status_string(qt2.QT2_ERR_BOUNDS).startswith("a kernel store")
+
+
 def test_built_for_sm100a_only():
     out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", qt2.LIB_PATH], capture_output=True,
                          text=True).stdout
@@ -40,7 +54,7 @@ def test_built_for_sm100a_only():
 
 def test_version_and_status_strings(L):
     assert qt2.qt2_version() >= 100
-    for code in range(0, -9, -1):
+    for code in range(0, -10, -1):
         s = qt2.qt2_status_string(code)
         assert s and s != "unknown status"
 
