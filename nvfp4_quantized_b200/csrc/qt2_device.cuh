@@ -39,7 +39,7 @@ __device__ __noinline__ bool store_in_bounds(const void *p, uint64_t bytes, cons
 #define QT2_STORE_OK(p, bytes, base, extent) \
     (::qt2::store_in_bounds((p), (uint64_t)(bytes), (base), (uint64_t)(extent)))
 #else
-#define QT2_STORE_OK(p, bytes, base, extent) true
+#define QT2_STORE_OK(p, bytes, base, extent) ((void)(p), (void)(bytes), (void)(base), (void)(extent), true)
 #endif
 
 // Upper bound of any single wait inside a kernel (ns).  A correct launch never comes close.
