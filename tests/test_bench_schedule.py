@@ -149,3 +149,18 @@ def test_onepass_quantizes_each_tensor_once_per_step_with_a_new_seed(config):
         assert {c[2] for c in calls} == {calls[0][2]}               # one seed for the whole step
         seeds.append(calls[0][2])
     assert len(set(seeds)) == len(seeds)
+
+
+def test_clock_reasons_that_force_a_second_measurement():
+    """The sampler's summary names the NVML clock-event reasons seen under load; hardware and
+    thermal slowdowns make the bench measure again, the power cap alone does not."""
+    c = bench.ClockSampler(0)
+    c.max_mhz = 1965
+    c.samples = [(1965, 600.0, 0x4), (1965, 620.0, 0x4), (1200, 10.0, 0x8)]   # the idle sample is ignored
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+    assert not set(s["reasons"]) & bench.THROTTLE_REASONS
+    c.samples = [(1965, 600.0, 0x4), (1700, 640.0, 0x4 | 0x40)]
+    s = c.summary()
+    assert set(s["reasons"]) == {"sw_power_cap", "hw_thermal_slowdown"}
+    assert set(s["reasons"]) & bench.THROTTLE_REASONS
