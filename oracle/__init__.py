@@ -331,6 +331,36 @@ def msedEN(x, seed: int, tid: int, view: str = "row") -> View:
     return View(codes, scales, g, amax=np.float32(A), P=P, S=S, amax_g=amax_g, signs=sgn)
 
 
+def msedEN_rows(x, rows, seed: int, tid: int, view: str = "row") -> View:
+    """Selected view rows of msedEN(x, seed, tid, view), for views too large to quantize whole
+    on the host: the view max A (every rotated value of the whole view, hence its tensor scale g)
+    is taken over all rows, then the MS-EDEN steps run on the selected rows only, each row's
+    scale draws keyed by its own view-row index as in the whole view.  Returns a View of
+    len(rows) rows (codes, scales, the whole view's g, and P, S, amax_g of those rows)."""
+    b = _bf16_bits(x)
+    if view == "col":
+        b = np.ascontiguousarray(b.T)
+    elif view != "row":
+        raise ValueError(view)
+    R, C = b.shape
+    sgn = rht_signs(seed)
+    A = float(rotated_amax(b, sgn))
+    if not np.isfinite(A):
+        raise ValueError("the rotated values overflow binary32 (|x| above about 2^121)")
+    g = lib().or_msedEN_tensor_scale(A)
+    rows = [int(r) for r in rows]
+    # whole-view buffers (zero pages; only the selected rows are touched)
+    codes = np.zeros((R, C // 2), np.uint8)
+    amax_g = np.zeros((R, C // 16), np.float32)
+    P = np.zeros((R, C // 16), np.float32)
+    S = np.zeros((R, C // 128), np.float32)
+    scales = np.zeros((R, C // 16), np.uint8)
+    for r in rows:
+        lib().or_msedEN_rows_stage1(_p(b), R, C, _p(sgn), r, r + 1, _p(codes), _p(amax_g), _p(P), _p(S))
+        lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r, r + 1, _p(scales))
+    return View(codes[rows], scales[rows], g, amax=np.float32(A), P=P[rows], S=S[rows], amax_g=amax_g[rows])
+
+
 def msedEN_rotated(y: np.ndarray, seed: int, tid: int) -> View:
     """The MS-EDEN steps on values that are already rotated (fp32 [R][C], C a multiple of 128),
     e.g. by a uniformly random orthogonal map instead of the randomized Hadamard: group scales,

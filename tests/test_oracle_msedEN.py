@@ -353,3 +353,19 @@ def test_scale_sr_outcomes_enumerated_on_one_128_block():
     nz = var > 0
     zc = (s1 / B - E0)[nz] / np.sqrt(var[nz] / B)
     assert np.max(np.abs(zc)) < thr
+
+
+def test_selected_rows_equal_the_whole_view():
+    """msedEN_rows (the view max over all rows, the steps on selected rows only) gives exactly
+    the selected rows of msedEN, both views: the view max, every code, scale and pre-scale."""
+    rng = np.random.default_rng(31)
+    xf = rng.standard_normal((384, 512)).astype(np.float32)
+    xf[200, 7] = 40.0                      # the view max sits outside the selected rows
+    x = _bf16(xf)
+    for view, rows in (("row", [0, 5, 127, 128, 383]), ("col", [1, 64, 300, 511])):
+        whole = O.msedEN(x, 13, 2, view)
+        part = O.msedEN_rows(x, rows, 13, 2, view)
+        assert part.g == whole.g and part.amax == whole.amax
+        assert np.array_equal(part.codes, whole.codes[rows])
+        assert np.array_equal(part.scales, whole.scales[rows])
+        assert np.array_equal(part.P, whole.P[rows]) and np.array_equal(part.S, whole.S[rows])
