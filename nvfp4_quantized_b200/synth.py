@@ -24,6 +24,8 @@ SHAPES = {
     "llm1p9b": (16384, 2048, 8192),
     "mlp8b_up": (16384, 4096, 14336),
     "mlp8b_down": (16384, 14336, 4096),
+    "stack1p1b_qkv": (32768, 2048, 6144),
+    "stack1p1b_down": (32768, 5632, 2048),
 }
 
 # Workloads made of several linear layers: (name, M, K, N, x kind, dY kind, name of the linear
@@ -45,7 +47,9 @@ STACKS = {
                   ("down", 32768, 5632, 2048, "silu_gated", "gauss_1e-4", None)],
 }
 _SINGLE_KINDS = {"tiny": ("gauss", "gauss1"), "llm1p9b": ("t3_outlier_channels", "gauss_1e-4"),
-                 "mlp8b_up": ("gauss", "lognormal_rows"), "mlp8b_down": ("silu_gated", "lognormal_rows")}
+                 "mlp8b_up": ("gauss", "lognormal_rows"), "mlp8b_down": ("silu_gated", "lognormal_rows"),
+                 "stack1p1b_qkv": ("t3_outlier_channels", "gauss_1e-4"),
+                 "stack1p1b_down": ("silu_gated", "gauss_1e-4")}
 
 
 def stack_linears(cfg: str):
@@ -136,26 +140,15 @@ def make_dy(M: int, N: int, kind: str, seed: int, device="cpu") -> torch.Tensor:
 
 
 def linear_inputs(cfg: str, seed: int = 0, device="cpu"):
-    """(X [M,K], W [N,K], dY [M,N]) bf16 for a named linear-layer workload."""
-    M, K, N = SHAPES[cfg]
-    if cfg == "tiny":
-        x = make_x(M, K, "gauss", seed, device)
-        w = make_w(N, K, seed + 1, std=0.02, device=device)
-        dy = make_dy(M, N, "gauss1", seed + 2, device)
-    elif cfg == "llm1p9b":
-        x = make_x(M, K, "t3_outlier_channels", seed, device)
-        w = make_w(N, K, seed + 1, device=device)
-        dy = make_dy(M, N, "gauss_1e-4", seed + 2, device)
-    elif cfg == "mlp8b_up":
-        x = make_x(M, K, "gauss", seed, device)
-        w = make_w(N, K, seed + 1, device=device)
-        dy = make_dy(M, N, "lognormal_rows", seed + 2, device)
-    elif cfg == "mlp8b_down":
-        x = make_x(M, K, "silu_gated", seed, device)
-        w = make_w(N, K, seed + 1, device=device)
-        dy = make_dy(M, N, "lognormal_rows", seed + 2, device)
-    else:
+    """(X [M,K], W [N,K], dY [M,N]) bf16 for a named linear-layer workload: X and dY of the
+    workload's kinds from sub-seeds seed and seed + 2, W ~ N(0, 0.02) from seed + 1."""
+    if cfg not in SHAPES:
         raise ValueError(cfg)
+    M, K, N = SHAPES[cfg]
+    xk, dk = _SINGLE_KINDS[cfg]
+    x = make_x(M, K, xk, seed, device)
+    w = make_w(N, K, seed + 1, device=device)
+    dy = make_dy(M, N, dk, seed + 2, device)
     return x, w, dy
 
 

@@ -82,7 +82,7 @@ def _full_view(view: qt2.View, R, C):
             np.float32(view.tensor_scale.item()))
 
 
-@pytest.mark.parametrize("config", ["llm1p9b", "mlp8b_up", "mlp8b_down"])
+@pytest.mark.parametrize("config", ["llm1p9b", "mlp8b_up", "mlp8b_down", "stack1p1b_qkv", "stack1p1b_down"])
 def test_full_size_views_and_layer(config):
     """Full-size layer in the launch configuration the benchmark times: EVERY code, scale and
     tensor scale of every quantized view (forward views of X and W, MS-EDEN views of dY both
