@@ -69,6 +69,7 @@ def lib():
                 "or_fwd46_sq_blocks": (None, [vp, i64, i64, f32, i64, i64, vp, vp, vp, vp, vp]),
                 "or_msedEN_rows_stage1": (None, [vp, i64, i64, vp, i64, i64, vp, vp, vp, vp]),
                 "or_msedEN_rotated_stage1": (None, [vp, i64, i64, i64, i64, vp, vp, vp, vp]),
+                "or_msedEN_rows_stage1_g16": (None, [vp, i64, i64, vp, i64, i64, vp, vp, vp]),
                 "or_msedEN_tensor_scale": (f32, [f32]),
                 "or_msedEN_finalize": (None, [vp, i64, i64, f32, u64, u32, i64, i64, vp]),
                 "or_dequant": (None, [vp, vp, i64, i64, f32, i64, i64, vp]),
@@ -329,6 +330,27 @@ def msedEN(x, seed: int, tid: int, view: str = "row") -> View:
     scales = np.zeros((R, C // 16), np.uint8)
     _rows(lambda r0, r1: lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r0, r1, _p(scales)), R)
     return View(codes, scales, g, amax=np.float32(A), P=P, S=S, amax_g=amax_g, signs=sgn)
+
+
+def msedEN_group16(x, seed: int, tid: int) -> View:
+    """Row view of MS-EDEN with the EDEN factor taken per 16-element group instead of per
+    128-element rotation block: the other reading of the grouping the pages leave open, kept to
+    compare the two (bias and error); the method itself is msedEN."""
+    b = _bf16_bits(x)
+    R, C = b.shape
+    sgn = rht_signs(seed)
+    codes = np.zeros((R, C // 2), np.uint8)
+    amax_g = np.zeros((R, C // 16), np.float32)
+    P = np.zeros((R, C // 16), np.float32)
+    _rows(lambda r0, r1: lib().or_msedEN_rows_stage1_g16(_p(b), R, C, _p(sgn), r0, r1, _p(codes), _p(amax_g),
+                                                         _p(P)), R)
+    A = float(amax_g.max()) if amax_g.size else 0.0
+    if not np.isfinite(A):
+        raise ValueError("the rotated values overflow binary32 (|x| above about 2^121)")
+    g = lib().or_msedEN_tensor_scale(A)
+    scales = np.zeros((R, C // 16), np.uint8)
+    _rows(lambda r0, r1: lib().or_msedEN_finalize(_p(P), R, C, g, seed, tid, r0, r1, _p(scales)), R)
+    return View(codes, scales, g, amax=np.float32(A), P=P, amax_g=amax_g, signs=sgn)
 
 
 def msedEN_rows(x, rows, seed: int, tid: int, view: str = "row") -> View:

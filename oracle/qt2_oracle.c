@@ -415,6 +415,54 @@ OR_EXPORT void or_msedEN_rows_stage1(const uint16_t *x, int64_t R, int64_t C, co
     }
 }
 
+/* The alternative EDEN grouping the pages leave open (one factor per 16-element group instead
+ * of per 128-element rotation block), kept only to compare the two readings: the same steps as
+ * or_eden_block with S_q = (sum y^2) / (p * sum val*y) over each group q alone.  Returns nothing
+ * per block; P[q] = S_q * p_q. */
+static void or_eden_group16(const float y[128], uint8_t codes[64], float amax_g[8], float P[8])
+{
+    uint8_t cq[128];
+    for (int q = 0; q < 8; q++) {
+        const float *yq = y + 16 * q;
+        float a = 0.0f;
+        for (int i = 0; i < 16; i++) if (fabsf(yq[i]) > a) a = fabsf(yq[i]);
+        amax_g[q] = a;
+        if (!(a >= OR_TINY)) {
+            P[q] = 0.0f;
+            for (int i = 0; i < 16; i++) cq[16 * q + i] = signbit(yq[i]) ? 8 : 0;
+            continue;
+        }
+        float p = a / 6.0f;
+        float rcp = 1.0f / p;
+        float tv[16], nv[16];
+        for (int i = 0; i < 16; i++) {
+            uint8_t c = or_e2m1_encode(yq[i] * rcp);
+            cq[16 * q + i] = c;
+            tv[i] = or_e2m1_value(c) * yq[i];
+            nv[i] = yq[i] * yq[i];
+        }
+        float num = or_tree(nv, 16), den = p * or_tree(tv, 16);
+        float S = den > 0.0f ? num / den : 1.0f;
+        P[q] = S * p;
+    }
+    for (int i = 0; i < 64; i++) codes[i] = (uint8_t)(cq[2 * i] | (cq[2 * i + 1] << 4));
+}
+
+/* Stage 1 with the per-16-group EDEN factor (comparison of readings only; not the method). */
+OR_EXPORT void or_msedEN_rows_stage1_g16(const uint16_t *x, int64_t R, int64_t C, const float sgn[128],
+                                         int64_t r0, int64_t r1, uint8_t *codes, float *amax_g, float *P)
+{
+    (void)R;
+    int64_t G = C / 16;
+    for (int64_t r = r0; r < r1; r++)
+        for (int64_t b = 0; b < C / 128; b++) {
+            float y[128];
+            for (int i = 0; i < 128; i++) y[i] = sgn[i] * or_bf16_to_f32(x[r * C + b * 128 + i]);
+            or_fwht128(y);
+            or_eden_group16(y, codes + r * (C / 2) + b * 64, amax_g + r * G + b * 8, P + r * G + b * 8);
+        }
+}
+
 /* The same EDEN steps on values already rotated by some other orthogonal map (fp32 [R][C], C a
  * multiple of 128): used to separate the EDEN steps' own unbiasedness from that of the
  * 128-point randomized Hadamard rotation (EDEN is exactly unbiased for a uniformly random
