@@ -19,7 +19,7 @@
  *     a negative qt2_status is returned.  Launch failures map to QT2_ERR_CUDA.  No call aborts.
  *   - bf16 matrices are row-major with a leading dimension `ld` (elements between rows,
  *     ld >= cols, ld a multiple of 8) and 16-byte aligned base pointers.
- *   - Every dimension must be a positive multiple of 128.
+ *   - Every dimension must be a positive multiple of 128, below 2^31.
  *   - The device must be compute capability 10.0 (B200); otherwise QT2_ERR_DEVICE.
  *   - Inputs must be finite.  A quantizer that meets inf or NaN in its input records
  *     QT2_ERR_NONFINITE in the device status word (qt2_device_status); what its outputs then

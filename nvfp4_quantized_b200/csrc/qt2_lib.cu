@@ -359,7 +359,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool dim_ok(int64_t d) { return d > 0 && d % 128 == 0 && d <= (int64_t(1) << 31); }
+// Dimensions reach the kernels as 32-bit ints (GEMM extents, TMA coordinates): below 2^31.
+bool dim_ok(int64_t d) { return d > 0 && d % 128 == 0 && d < (int64_t(1) << 31); }
 
 qt2_status check_device() {
     const int fa = fault_at("device");

@@ -76,6 +76,20 @@ def _view(codes=0x10000, scales=0x20000, ts=0x30000):
     return qt2.NVFP4ViewC(codes, scales, ts)
 
 
+def test_dimension_limit(L):
+    """Dimensions reach the kernels as 32-bit ints: 2^31 - 128 is accepted by the size queries,
+    2^31 is refused with QT2_ERR_SHAPE before any CUDA call."""
+    big = (1 << 31) - 128
+    assert qt2.qt2_quant_msedEN_workspace_size(big, 128, qt2.QT2_LAYOUT_ROW) > 0
+    for bad in (1 << 31, 1 << 32):
+        with pytest.raises(qt2.QT2Error) as e:
+            qt2.qt2_quant_msedEN_workspace_size(bad, 128, qt2.QT2_LAYOUT_ROW)
+        assert e.value.status == qt2.QT2_ERR_SHAPE
+        with pytest.raises(qt2.QT2Error) as e:
+            qt2.qt2_linear_fwd_workspace_size(128, bad, 128)
+        assert e.value.status == qt2.QT2_ERR_SHAPE
+
+
 def test_host_validation_codes(L):
     """Fake, never-dereferenced device addresses: validation happens before any CUDA call."""
     v = _view()
