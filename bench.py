@@ -710,10 +710,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=128)
     ap.add_argument("--ref-w-rows", type=int, default=2048)
-    ap.add_argument("--cpu-tokens", type=int, default=256)
-    ap.add_argument("--cpu-w-rows", type=int, default=4096)
-    ap.add_argument("--cpu-tokens-1t", type=int, default=128)
-    ap.add_argument("--cpu-w-rows-1t", type=int, default=1024)
+    # the oracle's samples: about 10 s of host work each (all cores; one thread)
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--cpu-w-rows", type=int, default=8192)
+    ap.add_argument("--cpu-tokens-1t", type=int, default=256)
+    ap.add_argument("--cpu-w-rows-1t", type=int, default=3072)
     ap.add_argument("--schedule", choices=["onepass", "separate", "fused", "local"], default="onepass",
                     help="onepass (default): every tensor quantized once a step, both of its views from one read "
                          "(qt2_quant_fwd46_msedEN_col on X and on W; MS-EDEN of dY, both views); separate: each "
