@@ -22,19 +22,6 @@
 
 namespace qt2 {
 
-template <int N>
-__device__ __forceinline__ float tree_sum(const float *v) {
-    float t[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) t[i] = v[i];
-#pragma unroll
-    for (int w = N; w > 1; w >>= 1) {
-#pragma unroll
-        for (int i = 0; i < w / 2; ++i) t[i] = __fadd_rn(t[2 * i], t[2 * i + 1]);
-    }
-    return t[0];
-}
-
 // ---------------------------------------------------------------------------------------------
 // Tensor max |x| of a bf16 matrix ([FAF]: global NVFP4 scales need the tensor-wide maximum).
 // Magnitudes of finite bf16 values order like their bit patterns with the sign cleared, so the
